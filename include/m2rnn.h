@@ -1,0 +1,120 @@
+/*
+ * m2rnn.h — C ABI of the B200 (sm_100a) M²RNN recurrence library (libm2rnn.so).
+ *
+ * The operation (per batch element b and head h, independently):
+ *   Z_t = tanh(H_{t-1} W + k_t v_tᵀ)
+ *   H_t = f_t H_{t-1} + (1 - f_t) Z_t
+ *   y_t = H_tᵀ q_t
+ * The first two lines are the state-update equations of "M²RNN: Non-Linear
+ * RNNs with Matrix-Valued States for Scalable Language Modeling"
+ * (gist.science technical summary, §2.1 core architecture design; also the
+ * wispaper.ai post "M2 RNN: Breaking the Expressivity Ceiling of Linear RNNs
+ * with Matrix-Valued States", §1 The Core Recurrence).  H_t is K×V, W is V×V
+ * per head (it right-multiplies H_{t-1}; §2.2 gives the GEMM shape (K, V, V)),
+ * f_t ∈ [0,1] is one scalar per (b, head, t) that depends on the input only.
+ * The readout y_t = H_tᵀ q_t (q_t ∈ R^K, applied to the updated state) is
+ * this library's reading: the pages define no readout.
+ *
+ * Layout: every tensor is dense, contiguous, head-first, row-major:
+ *   k, q   [B][H][T][K]      v, y, dy   [B][H][T][V]      f, df  [B][H][T]
+ *   W, dW  [H][V][V]         H0, HT, dHT, dH0  [B][H][K][V]
+ *   ckpt   [B][H][ceil(T/C)][K][V]   (C = ckpt_stride; ckpt[.,.,c] = H_{c·C})
+ * Element types: in M2RNN_MODE_BF16_TC the inputs k, v, q, W, dy are bf16
+ * (raw 16-bit words) and everything else is fp32.  In M2RNN_MODE_FP32_DEBUG
+ * all tensors are fp32.
+ *
+ * Ownership and synchronisation: the caller allocates every buffer (device
+ * memory) and the workspace; the library allocates nothing, keeps no state
+ * between calls and never synchronises, except in m2rnn_get_device_status.
+ * Calls are stream-ordered and asynchronous.  Outputs are overwritten, never
+ * accumulated (dW is the sum over batch and time, written once).  All
+ * pointers must be 16-byte aligned device pointers.
+ *
+ * Errors: argument problems return a status immediately and launch nothing.
+ * Launch failures return M2RNN_ERR_CUDA.  Every wait inside a kernel is
+ * bounded; a wait that runs out sets a status word in the workspace and the
+ * kernel returns early (its outputs are then undefined); read it with
+ * m2rnn_get_device_status.
+ */
+#ifndef M2RNN_H_
+#define M2RNN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    M2RNN_OK = 0,
+    M2RNN_ERR_INVALID_ARG = 1,       /* NULL required pointer, negative size, bad mode */
+    M2RNN_ERR_UNSUPPORTED_SHAPE = 2, /* K or V outside {16,32,64,128}, ckpt_stride < 1 */
+    M2RNN_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+    M2RNN_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than m2rnn_workspace_size */
+    M2RNN_ERR_CUDA = 5,              /* a CUDA runtime call or kernel launch failed */
+    M2RNN_ERR_DEVICE_TIMEOUT = 6     /* a bounded device-side wait ran out */
+} m2rnn_status;
+
+typedef enum {
+    /* bf16 k/v/q/W inputs; the per-step H_{t-1}·W runs on the tcgen05 tensor
+     * cores (bf16 operands, fp32 accumulation in tensor memory).  The fp32
+     * state is fed to the MMA as a compensated pair of bf16 operands
+     * (hi + lo), so the operand carries about 16 bits of mantissa. */
+    M2RNN_MODE_BF16_TC = 0,
+    /* fp32 everything, CUDA-core FFMA and accurate tanhf: a slow reference
+     * mode on the device. */
+    M2RNN_MODE_FP32_DEBUG = 1
+} m2rnn_mode;
+
+typedef struct {
+    int B, H, T, K, V;  /* batch, heads, steps, state rows (key dim), state columns (value dim) */
+    int mode;           /* m2rnn_mode */
+    int ckpt_stride;    /* C >= 1: the forward stores H_{c·C} for the backward */
+} m2rnn_dims;
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* m2rnn_stream_t;
+
+/* Bytes of device workspace a call needs (forward when backward == 0).
+ * Returns 0 for invalid dims.  The first 256 bytes hold the device status
+ * word: zero them once after allocating the workspace. */
+size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward);
+
+/* Forward scan.  H0 may be NULL (zero initial state).  HT (final state) and
+ * ckpt (checkpoints for m2rnn_backward) may be NULL.  y is required. */
+m2rnn_status m2rnn_forward(const m2rnn_dims* d,
+                           const void* k, const void* v, const void* q,
+                           const float* f, const void* W, const float* H0,
+                           float* y, float* HT, float* ckpt,
+                           void* workspace, size_t ws_bytes, m2rnn_stream_t stream);
+
+/* Backward through time for the loss L with dL/dy = dy and dL/dH_T = dHT
+ * (NULL = 0).  ckpt must come from m2rnn_forward with the same inputs and
+ * the same dims (including ckpt_stride); the states inside each chunk of C
+ * steps are recomputed from it.  Writes dk, dv, dq, df, dW, dH0 (all
+ * required, all fp32). */
+m2rnn_status m2rnn_backward(const m2rnn_dims* d,
+                            const void* k, const void* v, const void* q,
+                            const float* f, const void* W, const float* ckpt,
+                            const void* dy, const float* dHT,
+                            float* dk, float* dv, float* dq, float* df,
+                            float* dW, float* dH0,
+                            void* workspace, size_t ws_bytes, m2rnn_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the status word in `workspace`.
+ * Returns M2RNN_OK or M2RNN_ERR_DEVICE_TIMEOUT (or M2RNN_ERR_CUDA). */
+m2rnn_status m2rnn_get_device_status(void* workspace, m2rnn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* m2rnn_status_string(m2rnn_status s);
+
+/* Upper bound, in nanoseconds, for every device-side wait of later launches
+ * (default 2e9).  Values below 1e5 are raised to 1e5. */
+void m2rnn_set_wait_limit_ns(uint64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M2RNN_H_ */

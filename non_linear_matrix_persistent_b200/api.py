@@ -1,0 +1,148 @@
+"""Python binding of libm2rnn.so over torch tensors (argument marshalling only).
+
+Every step of the recurrence runs in the CUDA library; torch only provides
+device memory and the current stream.  Names follow include/m2rnn.h.
+
+  y, HT, ckpt = forward(k, v, q, f, W, H0=None, ckpt_stride=16, want_ckpt=False)
+  grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=16)
+
+bf16 k/v/q/W select the tensor-core mode (M2RNN_MODE_BF16_TC); fp32 select
+the fp32 debug mode.  Tensors must be contiguous CUDA tensors with the
+head-first layouts of the header.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import Dims, M2RNNError
+
+_workspaces: Dict[Tuple[int, int], torch.Tensor] = {}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _mode(k: torch.Tensor) -> int:
+    if k.dtype == torch.bfloat16:
+        return _lib.MODE_BF16_TC
+    if k.dtype == torch.float32:
+        return _lib.MODE_FP32_DEBUG
+    raise TypeError("k/v/q/W must be bfloat16 (tensor-core mode) or float32 (debug mode), got %s" % k.dtype)
+
+
+def _check(name, t, shape, dtype, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError("%s must be a CUDA tensor on %s" % (name, device))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype != dtype:
+        raise TypeError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16) -> Dims:
+    B, H, T, K = k.shape
+    return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride)
+
+
+def workspace(d: Dims, backward: bool, device) -> torch.Tensor:
+    """Zero-initialised device workspace (cached per device, grown on demand)."""
+    need = _lib.lib().m2rnn_workspace_size(d, 1 if backward else 0)
+    if need == 0:
+        raise M2RNNError(_lib.ERR_INVALID_ARG, "m2rnn_workspace_size")
+    key = (device.index if device.index is not None else torch.cuda.current_device(), 0)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def num_checkpoints(T: int, ckpt_stride: int) -> int:
+    return (T + ckpt_stride - 1) // ckpt_stride
+
+
+def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = False,
+            want_HT: bool = True, out: Optional[dict] = None):
+    """Runs the forward scan.  Returns (y, HT or None, ckpt or None)."""
+    dev = k.device
+    d = dims_of(k, v, ckpt_stride)
+    B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
+    lp = k.dtype
+    _check("k", k, (B, H, T, K), lp, dev)
+    _check("v", v, (B, H, T, V), lp, dev)
+    _check("q", q, (B, H, T, K), lp, dev)
+    _check("f", f, (B, H, T), torch.float32, dev)
+    _check("W", W, (H, V, V), lp, dev)
+    _check("H0", H0, (B, H, K, V), torch.float32, dev)
+    out = out or {}
+    y = out.get("y")
+    if y is None:
+        y = torch.empty(B, H, T, V, dtype=torch.float32, device=dev)
+    HT = out.get("HT") if want_HT else None
+    if want_HT and HT is None:
+        HT = torch.empty(B, H, K, V, dtype=torch.float32, device=dev)
+    ckpt = out.get("ckpt") if want_ckpt else None
+    if want_ckpt and ckpt is None:
+        ckpt = torch.empty(B, H, num_checkpoints(T, ckpt_stride), K, V, dtype=torch.float32, device=dev)
+    ws = workspace(d, False, dev)
+    st = _lib.lib().m2rnn_forward(d, _ptr(k), _ptr(v), _ptr(q), _ptr(f), _ptr(W), _ptr(H0), _ptr(y), _ptr(HT),
+                                  _ptr(ckpt), _ptr(ws), ws.numel(), _stream(dev))
+    if st != _lib.OK:
+        raise M2RNNError(st, "m2rnn_forward")
+    return y, HT, ckpt
+
+
+def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: Optional[dict] = None):
+    """BPTT from the forward's checkpoints.  Returns dict dk, dv, dq, df, dW, dH0 (fp32)."""
+    dev = k.device
+    d = dims_of(k, v, ckpt_stride)
+    B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
+    lp = k.dtype
+    _check("k", k, (B, H, T, K), lp, dev)
+    _check("v", v, (B, H, T, V), lp, dev)
+    _check("q", q, (B, H, T, K), lp, dev)
+    _check("f", f, (B, H, T), torch.float32, dev)
+    _check("W", W, (H, V, V), lp, dev)
+    _check("ckpt", ckpt, (B, H, num_checkpoints(T, ckpt_stride), K, V), torch.float32, dev)
+    _check("dy", dy, (B, H, T, V), lp, dev)
+    _check("dHT", dHT, (B, H, K, V), torch.float32, dev)
+    out = dict(out or {})
+    shapes = {"dk": (B, H, T, K), "dv": (B, H, T, V), "dq": (B, H, T, K), "df": (B, H, T),
+              "dW": (H, V, V), "dH0": (B, H, K, V)}
+    for n, s in shapes.items():
+        if out.get(n) is None:
+            out[n] = torch.empty(*s, dtype=torch.float32, device=dev)
+    ws = workspace(d, True, dev)
+    st = _lib.lib().m2rnn_backward(d, _ptr(k), _ptr(v), _ptr(q), _ptr(f), _ptr(W), _ptr(ckpt), _ptr(dy),
+                                   _ptr(dHT), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dq"]), _ptr(out["df"]),
+                                   _ptr(out["dW"]), _ptr(out["dH0"]), _ptr(ws), ws.numel(), _stream(dev))
+    if st != _lib.OK:
+        raise M2RNNError(st, "m2rnn_backward")
+    return out
+
+
+def device_status(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device status of the cached workspace."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    key = (dev.index if dev.index is not None else torch.cuda.current_device(), 0)
+    ws = _workspaces.get(key)
+    if ws is None:
+        return _lib.OK
+    return _lib.lib().m2rnn_get_device_status(_ptr(ws), _stream(dev))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _lib.lib().m2rnn_set_wait_limit_ns(int(ns))

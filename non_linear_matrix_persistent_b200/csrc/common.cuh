@@ -1,0 +1,74 @@
+// Shared device-side pieces of the M²RNN kernels: launch parameters, the
+// device status word and bounded mbarrier waits.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+
+namespace m2rnn {
+
+// Device status codes written into the workspace status word.
+enum : uint32_t {
+    kDevOk = 0,
+    kDevTimeout = 1u,
+};
+
+struct Params {
+    int B, H, T, K, V, C;
+    const void* k;
+    const void* v;
+    const void* q;
+    const float* f;
+    const void* W;
+    const float* H0;    // forward: initial state (may be null)
+    float* y;
+    float* HT;          // may be null
+    float* ckpt;        // forward: checkpoint output (may be null); backward: input
+    // backward
+    const void* dy;
+    const float* dHT;   // may be null
+    float* dk;
+    float* dv;
+    float* dq;
+    float* df;
+    float* dW;
+    float* dH0;
+    float* dW_part;     // [B*H][V][V] partial dW (workspace)
+    float* scratch;     // per-CTA recompute scratch (workspace)
+    uint32_t* status;   // device status word (workspace)
+    uint64_t wait_limit_ns;
+};
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the CTA-wide
+// abort flag and the device status word) when the wait runs longer than the
+// limit, or when another thread of the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  const Params& p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+            *abort_flag = 1;
+            atomicOr(p.status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// Same, but ignores the abort flag (used to drain copies/MMAs in flight
+// before the CTA exits).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, const Params& p) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+            atomicOr(p.status, kDevTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+}  // namespace m2rnn

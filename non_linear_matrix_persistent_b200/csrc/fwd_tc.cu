@@ -1,0 +1,427 @@
+// M²RNN forward scan on the sm_100a tensor cores (tcgen05).
+//
+// Recurrence (gist.science technical summary of "M²RNN: Non-Linear RNNs with
+// Matrix-Valued States for Scalable Language Modeling", §2.1):
+//   Z_t = tanh(H_{t-1} W + k_t v_tᵀ),  H_t = f_t H_{t-1} + (1 - f_t) Z_t,
+// plus the readout y_t = H_tᵀ q_t (this library's reading; the pages define
+// none).  The pages parallelise the forward over batch × head with each SM
+// owning independent matrix states (§2.2); here one CTA owns one (b, h) pair
+// for all T steps, with the fp32 state in registers.
+//
+// Formulation.  The kernel computes the transpose of the transition GEMM,
+//   D = Wᵀ · H_{t-1}ᵀ   (M = V columns of H, N = state rows, contraction V),
+// so that tensor-memory lane j holds column j of H_{t-1}W.  Each epilogue
+// thread therefore owns one column j of the state and a block of its rows:
+// the rank-1 term k_t[i] v_t[j], the tanh, the gate blend and the readout
+// y_t[j] = Σ_i q_t[i] H_t[i, j] are all thread-local (the readout needs one
+// shuffle when a column is split over two half-warps).
+//
+//   A = Wᵀ      : shared memory, K-major, loaded once (bf16).
+//   B = H_{t-1}ᵀ: shared memory, MN-major, rewritten each step by the
+//                 epilogue.  The fp32 state is passed as a compensated pair
+//                 hi + lo of bf16 operands (hi = the top 16 bits of the fp32
+//                 word, lo = bf16(x - hi)), stacked along N, so one MMA
+//                 produces both products and the epilogue adds them.
+//   D           : tensor memory (fp32).
+//
+// The state rows of a pair are split into P = 2 tiles that alternate
+// (ping-pong): while the epilogue warpgroup of one tile runs tanh and the
+// blend, the tensor core computes the other tile's product.
+//
+// Warp roles: warps [0, 4P) epilogue (warp w serves tile w/4 and TMEM lane
+// quarter w%4), then one bulk-copy producer warp (k, q, v and f for TC steps
+// per ring stage), one MMA warp (also owns the TMEM allocation) and one
+// storer warp that sums the per-tile partial readouts and writes y.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace m2rnn {
+
+template <int K_, int V_>
+struct FwdTcCfg {
+    static constexpr int K = K_, V = V_;
+    static constexpr int P = 2;
+    static constexpr int MPAD = V <= 64 ? 64 : 128;
+    static constexpr int R = K / P;                       // state rows per tile
+    static constexpr int NT = 2 * R;                      // MMA N per tile (hi rows, then lo rows)
+    static constexpr int RT = (MPAD == 64) ? R / 2 : R;   // rows per epilogue thread
+    static constexpr int CH = RT < 32 ? RT : 32;          // rows per tensor-memory load
+    static constexpr int TC = 16;                         // steps per ring stage
+    static constexpr int S = 4;                           // ring stages
+    static constexpr int NWE = 4 * P;                     // epilogue warps
+    static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
+    static constexpr int NTHREADS = (NWE + 3) * 32;
+
+    static constexpr int A_BYTES = MPAD * V * 2;
+    static constexpr int B_BYTES = NT * V * 2;
+    static constexpr int ST_K = 0;
+    static constexpr int ST_Q = TC * K * 2;
+    static constexpr int ST_V = 2 * TC * K * 2;
+    static constexpr int ST_F = ST_V + TC * V * 2;
+    static constexpr int STAGE_BYTES = ((ST_F + TC * 4) + 127) / 128 * 128;
+    static constexpr int YBUF_BYTES = P * TC * V * 4;
+
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + A_BYTES;
+    static constexpr int OFF_RING = OFF_B + P * B_BYTES;
+    static constexpr int OFF_Y = OFF_RING + S * STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_Y + 2 * YBUF_BYTES;
+    static constexpr int NBAR = 2 * S + 2 * P + 4;
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
+    static constexpr int TMEM_COLS = (P * NT <= 32) ? 32 : (P * NT <= 64) ? 64 : (P * NT <= 128) ? 128 : 256;
+
+    static_assert(K % (2 * P) == 0 && RT >= 4 && RT % 4 == 0, "unsupported K");
+    static_assert((MPAD == 64 && NT % 8 == 0) || (MPAD == 128 && NT % 16 == 0), "bad MMA N");
+    static_assert(NT <= 256 && V % 16 == 0, "bad shape");
+    static_assert(RT % CH == 0, "chunking");
+    static_assert(SMEM_BYTES <= 227 * 1024, "smem");
+};
+
+// Loads n bf16 values (n = 4 or a multiple of 8; 8- or 16-byte aligned) from shared memory.
+template <int N>
+__device__ __forceinline__ void lds_bf16(const uint16_t* src, float (&out)[N]) {
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < N / 8; ++g) {
+            const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * g);
+            out[8 * g + 0] = bf16lo_to_f32(w.x); out[8 * g + 1] = bf16hi_to_f32(w.x);
+            out[8 * g + 2] = bf16lo_to_f32(w.y); out[8 * g + 3] = bf16hi_to_f32(w.y);
+            out[8 * g + 4] = bf16lo_to_f32(w.z); out[8 * g + 5] = bf16hi_to_f32(w.z);
+            out[8 * g + 6] = bf16lo_to_f32(w.w); out[8 * g + 7] = bf16hi_to_f32(w.w);
+        }
+    } else {
+        static_assert(N == 4, "lds_bf16");
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        out[0] = bf16lo_to_f32(w.x); out[1] = bf16hi_to_f32(w.x);
+        out[2] = bf16lo_to_f32(w.y); out[3] = bf16hi_to_f32(w.y);
+    }
+}
+
+// hi / lo bf16 pair of two fp32 values, packed two per 32-bit word
+// (element with the lower index in the low half).
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+    hi = __byte_perm(b0, b1, 0x7632);
+    const float l0 = x0 - __uint_as_float(b0 & 0xFFFF0000u);
+    const float l1 = x1 - __uint_as_float(b1 & 0xFFFF0000u);
+    const __nv_bfloat162 lp = __floats2bfloat162_rn(l0, l1);
+    lo = *reinterpret_cast<const uint32_t*>(&lp);
+}
+
+// Writes this thread's RT state values of column j into the MN-major B
+// operand of its tile: element (k = j, n) lives at
+//   (j/8)·(NT·16) + (n/8)·128 + (j%8)·16 + (n%8)·2,
+// hi values at n = nloc + r, lo values at n = R + nloc + r.
+template <class C>
+__device__ __forceinline__ void write_state_operand(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
+    uint8_t* colbase = Bt + (j >> 3) * (C::NT * 16) + (j & 7) * 16;
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g) {
+            uint4 hi, lo;
+            split_pack(h[8 * g + 0], h[8 * g + 1], hi.x, lo.x);
+            split_pack(h[8 * g + 2], h[8 * g + 3], hi.y, lo.y);
+            split_pack(h[8 * g + 4], h[8 * g + 5], hi.z, lo.z);
+            split_pack(h[8 * g + 6], h[8 * g + 7], hi.w, lo.w);
+            const int n = nloc + 8 * g;
+            *reinterpret_cast<uint4*>(colbase + (n >> 3) * 128) = hi;
+            *reinterpret_cast<uint4*>(colbase + ((C::R + n) >> 3) * 128) = lo;
+        }
+    } else {
+        uint2 hi, lo;
+        split_pack(h[0], h[1], hi.x, lo.x);
+        split_pack(h[2], h[3], hi.y, lo.y);
+        const int n = nloc;
+        *reinterpret_cast<uint2*>(colbase + (n >> 3) * 128 + (n & 7) * 2) = hi;
+        *reinterpret_cast<uint2*>(colbase + ((C::R + n) >> 3) * 128 + ((C::R + n) & 7) * 2) = lo;
+    }
+}
+
+template <int K, int V>
+__global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
+    using C = FwdTcCfg<K, V>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int hd = bh % p.H;
+    const int T = p.T;
+    const int nchunks = (T + C::TC - 1) / C::TC;
+    const int nck = (T + p.C - 1) / p.C;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    auto in_full = [&](int s) { return bar(s); };
+    auto in_empty = [&](int s) { return bar(C::S + s); };
+    auto bready = [&](int t) { return bar(2 * C::S + t); };
+    auto accfull = [&](int t) { return bar(2 * C::S + C::P + t); };
+    auto ypfull = [&](int i) { return bar(2 * C::S + 2 * C::P + i); };
+    auto ypempty = [&](int i) { return bar(2 * C::S + 2 * C::P + 2 + i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::S; ++s) {
+            mbar_init(in_full(s), 1);
+            mbar_init(in_empty(s), C::NWE);
+        }
+        for (int t = 0; t < C::P; ++t) {
+            mbar_init(bready(t), 4);
+            mbar_init(accfull(t), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(ypfull(i), C::NWE);
+            mbar_init(ypempty(i), 1);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    // A = Wᵀ (K-major, no swizzle): element (m = j, k = l) = W[l][j] at
+    // (j/8)·(V·16) + (l/8)·128 + (j%8)·16 + (l%8)·2; rows j >= V are zero.
+    {
+        const uint16_t* Wg = static_cast<const uint16_t*>(p.W) + (size_t)hd * V * V;
+        for (int idx = threadIdx.x; idx < C::MPAD * V; idx += C::NTHREADS) {
+            const int l = idx / C::MPAD, j = idx % C::MPAD;
+            const uint16_t w = (j < V) ? Wg[l * V + j] : (uint16_t)0;
+            *reinterpret_cast<uint16_t*>(smem + C::OFF_A + (j >> 3) * (V * 16) + (l >> 3) * 128 + (j & 7) * 16 +
+                                         (l & 7) * 2) = w;
+        }
+    }
+    fence_proxy_async_smem();
+    if (warp == C::W_MMA) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < C::NWE) {
+        // ------------------------------------------------------------ epilogue
+        const int tile = warp >> 2, qd = warp & 3;
+        const int half = (C::MPAD == 64) ? (lane >> 4) : 0;
+        const int j = (C::MPAD == 64) ? qd * 16 + (lane & 15) : qd * 32 + lane;
+        const bool jv = j < V;
+        const int nloc = half * C::RT;            // first row within the tile
+        const int row0 = tile * C::R + nloc;      // first state row
+        const size_t sbase = (size_t)bh * K * V;
+        uint8_t* Bt = smem + C::OFF_B + tile * C::B_BYTES;
+
+        float h[C::RT];
+#pragma unroll
+        for (int r = 0; r < C::RT; ++r) h[r] = (p.H0 != nullptr && jv) ? p.H0[sbase + (size_t)(row0 + r) * V + j] : 0.f;
+        if (p.ckpt != nullptr && jv) {
+            float* ck = p.ckpt + (size_t)bh * nck * K * V;
+#pragma unroll
+            for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
+        }
+        if (jv) write_state_operand<C>(Bt, h, j, nloc);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bready(tile));
+
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT);
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            const int c = t / C::TC, tt = t - c * C::TC, s = c % C::S;
+            const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            if (tt == 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (c / C::S) & 1, abort_flag, p));
+                if (ok && c >= 2)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), t & 1, abort_flag, p));
+            if (!ok) break;
+            tc_fence_after();
+
+            const float vj = jv ? bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + tt * V * 2 + j * 2))
+                                : 0.f;
+            const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
+            const uint16_t* kt = reinterpret_cast<const uint16_t*>(st + C::ST_K + tt * K * 2) + row0;
+#pragma unroll
+            for (int c0 = 0; c0 < C::RT; c0 += C::CH) {
+                uint32_t ahi[C::CH], alo[C::CH];
+                if constexpr (C::MPAD == 64) {
+                    tmem_ld_16x32bx2<C::CH, C::CH>(tbase + c0, ahi);
+                    tmem_ld_16x32bx2<C::CH, C::CH>(tbase + C::R + c0, alo);
+                } else {
+                    tmem_ld_32x32b<C::CH>(tbase + c0, ahi);
+                    tmem_ld_32x32b<C::CH>(tbase + C::R + c0, alo);
+                }
+                float kk[C::CH];
+                lds_bf16<C::CH>(kt + c0, kk);
+                tc_wait_ld();
+                reg_fence(ahi);
+                reg_fence(alo);
+#pragma unroll
+                for (int r = 0; r < C::CH; ++r) {
+                    float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
+                    a = fmaf(kk[r], vj, a);
+                    const float z = tanh_approx(a);
+                    h[c0 + r] = fmaf(g, z - h[c0 + r], h[c0 + r]);
+                }
+            }
+            tc_fence_before();
+            if (t + 1 < T) {
+                if (jv) write_state_operand<C>(Bt, h, j, nloc);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bready(tile));
+            }
+            // readout partial over this thread's rows (off the critical path)
+            {
+                float qq[C::RT];
+                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_Q + tt * K * 2) + row0, qq);
+                float yp = 0.f;
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) yp = fmaf(qq[r], h[r], yp);
+                if constexpr (C::MPAD == 64) yp += __shfl_xor_sync(0xffffffffu, yp, 16);
+                if (half == 0 && jv)
+                    reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES)[(tile * C::TC + tt) * V + j] = yp;
+            }
+            if (p.ckpt != nullptr && jv && (t + 1) < T && ((t + 1) % p.C) == 0) {
+                float* ck = p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * K * V;
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
+            }
+            if (tt == C::TC - 1 || t == T - 1) {
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(in_empty(s));
+                    mbar_arrive(ypfull(c & 1));
+                }
+            }
+        }
+        if (ok && p.HT != nullptr && jv) {
+#pragma unroll
+            for (int r = 0; r < C::RT; ++r) p.HT[sbase + (size_t)(row0 + r) * V + j] = h[r];
+        }
+    } else if (warp == C::W_PROD) {
+        // ------------------------------------------------------------ producer
+        int last = -1;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % C::S;
+            if (c >= C::S) {
+                const bool ok =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(in_empty(s), ((c / C::S) - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            const int t0 = c * C::TC, nt = min(C::TC, T - t0);
+            uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            if (lane < nt) reinterpret_cast<float*>(st + C::ST_F)[lane] = p.f[(size_t)bh * T + t0 + lane];
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t kb = (uint32_t)(nt * K * 2), vb = (uint32_t)(nt * V * 2);
+                mbar_arrive_expect_tx(in_full(s), 2 * kb + vb);
+                bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + ((size_t)bh * T + t0) * K, kb,
+                         in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + ((size_t)bh * T + t0) * K, kb,
+                         in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + ((size_t)bh * T + t0) * V, vb,
+                         in_full(s));
+            }
+            last = c;
+        }
+        // copies still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int c = max(0, last - C::S + 1); c <= last; ++c) mbar_wait_drain(in_full(c % C::S), (c / C::S) & 1, p);
+        __syncwarp();
+    } else if (warp == C::W_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(C::MPAD, C::NT, 0, 1);
+            const uint32_t a0 = smem_u32(smem + C::OFF_A);
+            int issued[C::P];
+#pragma unroll
+            for (int i = 0; i < C::P; ++i) issued[i] = -1;
+            bool ok = true;
+            for (int t = 0; t < T && ok; ++t) {
+#pragma unroll
+                for (int tile = 0; tile < C::P; ++tile) {
+                    if (!mbar_wait_bounded(bready(tile), t & 1, abort_flag, p)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t b0 = smem_u32(smem + C::OFF_B + tile * C::B_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < V / 16; ++ks) {
+                        const uint64_t ad = smem_desc(a0 + ks * 256, 128, V * 16);
+                        const uint64_t bd = smem_desc(b0 + ks * 2 * C::NT * 16, C::NT * 16, 128);
+                        tc_mma_f16_ss(tmem + tile * C::NT, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(accfull(tile));
+                    issued[tile] = t;
+                }
+            }
+#pragma unroll
+            for (int tile = 0; tile < C::P; ++tile)
+                if (issued[tile] >= 0) mbar_wait_drain(accfull(tile), issued[tile] & 1, p);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ y storer
+        for (int c = 0; c < nchunks; ++c) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(ypfull(c & 1), (c >> 1) & 1, abort_flag, p));
+            if (!ok) break;
+            const int t0 = c * C::TC, nt = min(C::TC, T - t0);
+            const float* yb = reinterpret_cast<const float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES);
+            float* yg = p.y + ((size_t)bh * T + t0) * V;
+            for (int e = lane * 4; e < nt * V; e += 128) {
+                float4 a = *reinterpret_cast<const float4*>(yb + e);
+#pragma unroll
+                for (int tile = 1; tile < C::P; ++tile) {
+                    const float4 b = *reinterpret_cast<const float4*>(yb + tile * C::TC * V + e);
+                    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+                }
+                *reinterpret_cast<float4*>(yg + e) = a;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ypempty(c & 1));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::W_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int K, int V>
+static cudaError_t launch_fwd_tc_kv(const Params& p, cudaStream_t stream) {
+    using C = FwdTcCfg<K, V>;
+    auto kern = m2rnn_fwd_tc_kernel<K, V>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<p.B * p.H, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <int K>
+static cudaError_t launch_fwd_tc_k(const Params& p, cudaStream_t s) {
+    switch (p.V) {
+        case 16: return launch_fwd_tc_kv<K, 16>(p, s);
+        case 32: return launch_fwd_tc_kv<K, 32>(p, s);
+        case 64: return launch_fwd_tc_kv<K, 64>(p, s);
+        case 128: return launch_fwd_tc_kv<K, 128>(p, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_fwd_tc(const Params& p, cudaStream_t s) {
+    switch (p.K) {
+        case 16: return launch_fwd_tc_k<16>(p, s);
+        case 32: return launch_fwd_tc_k<32>(p, s);
+        case 64: return launch_fwd_tc_k<64>(p, s);
+        case 128: return launch_fwd_tc_k<128>(p, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace m2rnn

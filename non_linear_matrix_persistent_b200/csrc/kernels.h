@@ -1,0 +1,24 @@
+// Host-side launchers of the M²RNN kernels (internal to libm2rnn.so).
+#pragma once
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace m2rnn {
+
+// tcgen05 forward scan (bf16 inputs).  K, V in {16, 32, 64, 128}.
+cudaError_t launch_fwd_tc(const Params& p, cudaStream_t s);
+// fp32 CUDA-core forward (debug mode).
+cudaError_t launch_fwd_fp32(const Params& p, cudaStream_t s);
+// fp32 CUDA-core backward (debug mode): chunked recompute + BPTT + dW reduce.
+cudaError_t launch_bwd_fp32(const Params& p, cudaStream_t s);
+// tcgen05 backward (bf16 inputs): chunked recompute + BPTT + dW reduce.
+cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s);
+// Deterministic dW[h] = sum_b dW_part[b, h] (fixed ascending order).
+cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
+
+// Workspace bytes beyond the 256-byte status header.
+size_t bwd_fp32_workspace(int B, int H, int K, int V, int C);
+size_t bwd_tc_workspace(int B, int H, int K, int V, int C);
+
+}  // namespace m2rnn

@@ -1,0 +1,88 @@
+"""Host-only checks of the C ABI (include/m2rnn.h): the library loads, exports
+every declared entry point, sizes workspaces and rejects bad arguments before
+touching the device.  No kernel is launched here."""
+import ctypes
+import re
+import os
+
+import pytest
+
+from non_linear_matrix_persistent_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def test_exports_match_header(L):
+    header = open(os.path.join(ROOT, "include", "m2rnn.h")).read()
+    declared = set(re.findall(r"\b(m2rnn_[a-z_]+)\s*\(", header))
+    assert declared == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16):
+    return _lib.Dims(B, H, T, K, V, mode, C)
+
+
+def test_workspace_size(L):
+    d = _dims()
+    assert L.m2rnn_workspace_size(d, 0) == 256
+    assert L.m2rnn_workspace_size(_dims(mode=1), 1) > 256
+    assert L.m2rnn_workspace_size(_dims(K=48), 0) == 0
+    assert L.m2rnn_workspace_size(_dims(mode=7), 0) == 0
+    assert L.m2rnn_workspace_size(None, 0) == 0
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert _lib.status_string(s).startswith("M2RNN_")
+    assert _lib.status_string(99) == "M2RNN_ERR_UNKNOWN"
+
+
+def _fwd(L, d, ptrs=None, ws_bytes=1 << 20):
+    p = dict(k=4096, v=4096, q=4096, f=4096, W=4096, H0=None, y=4096, HT=None, ckpt=None, ws=4096)
+    p.update(ptrs or {})
+    return L.m2rnn_forward(d, p["k"], p["v"], p["q"], p["f"], p["W"], p["H0"], p["y"], p["HT"], p["ckpt"],
+                           p["ws"], ws_bytes, None)
+
+
+def test_forward_argument_errors(L):
+    # every case fails validation, so nothing reaches the device
+    assert _fwd(L, None) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(K=24)) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(L, _dims(V=256)) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(L, _dims(C=0)) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(L, _dims(B=-1)) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(mode=3)) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(), {"k": None}) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(), {"y": None}) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(), {"ws": None}) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(), {"q": 4100}) == _lib.ERR_MISALIGNED
+    assert _fwd(L, _dims(), {"HT": 4104}) == _lib.ERR_MISALIGNED
+    assert _fwd(L, _dims(), ws_bytes=100) == _lib.ERR_WORKSPACE
+    # zero-sized batch: nothing to do
+    assert _fwd(L, _dims(B=0)) == _lib.OK
+
+
+def test_backward_argument_errors(L):
+    def bwd(d, **kw):
+        p = dict(k=4096, v=4096, q=4096, f=4096, W=4096, ckpt=4096, dy=4096, dHT=None, dk=4096, dv=4096,
+                 dq=4096, df=4096, dW=4096, dH0=4096, ws=4096, ws_bytes=1 << 40)
+        p.update(kw)
+        return L.m2rnn_backward(d, p["k"], p["v"], p["q"], p["f"], p["W"], p["ckpt"], p["dy"], p["dHT"], p["dk"],
+                                p["dv"], p["dq"], p["df"], p["dW"], p["dH0"], p["ws"], p["ws_bytes"], None)
+    assert bwd(_dims(), ckpt=None) == _lib.ERR_INVALID_ARG
+    assert bwd(_dims(), dW=None) == _lib.ERR_INVALID_ARG
+    assert bwd(_dims(), dy=4097) == _lib.ERR_MISALIGNED
+    assert bwd(_dims(mode=1), ws_bytes=256) == _lib.ERR_WORKSPACE
+    assert bwd(_dims(K=8)) == _lib.ERR_UNSUPPORTED_SHAPE
+
+
+def test_status_query_rejects_null(L):
+    assert L.m2rnn_get_device_status(None, None) == _lib.ERR_INVALID_ARG
