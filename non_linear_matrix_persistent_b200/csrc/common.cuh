@@ -43,12 +43,15 @@ struct Params {
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA-wide
 // abort flag and the device status word) when the wait runs longer than the
 // limit, or when another thread of the CTA has already aborted.
+// SPIN = true polls with test_wait (no suspension: lowest wake-up latency,
+// but the waiting warp keeps issuing).
+template <bool SPIN = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                   const Params& p) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (SPIN ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (SPIN ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > p.wait_limit_ns) {
             *abort_flag = 1;

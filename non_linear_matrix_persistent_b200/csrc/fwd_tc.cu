@@ -24,14 +24,20 @@
 //                 produces both products and the epilogue adds them.
 //   D           : tensor memory (fp32).
 //
-// The state rows of a pair are split into P = 2 tiles that alternate
-// (ping-pong): while the epilogue warpgroup of one tile runs tanh and the
-// blend, the tensor core computes the other tile's product.
+// Latency structure (measured on B200): a tcgen05.mma costs at least ~50-70
+// cycles, and issue -> commit -> mbarrier wake-up adds ~400 cycles, so a
+// step is bound by that round trip plus the epilogue, not by tensor
+// throughput.  The state rows of a pair are therefore split into P = 2 tiles
+// whose chains run concurrently (ping-pong): while the epilogue warps of one
+// tile run tanh and the blend, the tensor core computes the other tile's
+// product.  Two warps per TMEM lane quarter serve each tile (when the tile
+// has enough rows), so that each thread handles few rows.
 //
-// Warp roles: warps [0, 4P) epilogue (warp w serves tile w/4 and TMEM lane
-// quarter w%4), then one bulk-copy producer warp (k, q, v and f for TC steps
-// per ring stage), one MMA warp (also owns the TMEM allocation) and one
-// storer warp that sums the per-tile partial readouts and writes y.
+// Warp roles: warps [0, P·WPT) epilogue (warp w serves tile w / WPT, TMEM
+// lane quarter w % 4 and row group (w % WPT) / 4), then one bulk-copy
+// producer warp (k, q, v and f for TC steps per ring stage), one MMA warp
+// (also owns the TMEM allocation) and one storer warp that sums the partial
+// readouts and writes y.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -46,13 +52,19 @@ struct FwdTcCfg {
     static constexpr int MPAD = V <= 64 ? 64 : 128;
     static constexpr int R = K / P;                       // state rows per tile
     static constexpr int NT = 2 * R;                      // MMA N per tile (hi rows, then lo rows)
-    static constexpr int RT = (MPAD == 64) ? R / 2 : R;   // rows per epilogue thread
-    static constexpr int CH = RT < 32 ? RT : 32;          // rows per tensor-memory load
+    // row groups per tile served by separate warps of the same lane quarter
+    // (measured: helps the 128-column case, where a thread otherwise owns 64
+    // rows, and slightly hurts the 64-column case)
+    static constexpr int SUBS = (MPAD == 128) ? 2 : 1;
+    static constexpr int WPT = 4 * SUBS;                  // epilogue warps per tile
+    static constexpr int RT = (MPAD == 64) ? R / (2 * SUBS) : R / SUBS;  // rows per thread
+    static constexpr int CH = RT < 16 ? RT : 16;          // rows per tensor-memory load
     static constexpr int TC = 16;                         // steps per ring stage
     static constexpr int S = 4;                           // ring stages
-    static constexpr int NWE = 4 * P;                     // epilogue warps
+    static constexpr int NWE = P * WPT;                   // epilogue warps
     static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
     static constexpr int NTHREADS = (NWE + 3) * 32;
+    static constexpr int NSLOT = P * SUBS;                // readout partials per (t, j)
 
     static constexpr int A_BYTES = MPAD * V * 2;
     static constexpr int B_BYTES = NT * V * 2;
@@ -61,7 +73,7 @@ struct FwdTcCfg {
     static constexpr int ST_V = 2 * TC * K * 2;
     static constexpr int ST_F = ST_V + TC * V * 2;
     static constexpr int STAGE_BYTES = ((ST_F + TC * 4) + 127) / 128 * 128;
-    static constexpr int YBUF_BYTES = P * TC * V * 4;
+    static constexpr int YBUF_BYTES = NSLOT * TC * V * 4;
 
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + A_BYTES;
@@ -73,6 +85,7 @@ struct FwdTcCfg {
     static constexpr int TMEM_COLS = (P * NT <= 32) ? 32 : (P * NT <= 64) ? 64 : (P * NT <= 128) ? 128 : 256;
 
     static_assert(K % (2 * P) == 0 && RT >= 4 && RT % 4 == 0, "unsupported K");
+    static_assert(NTHREADS <= 1024, "block size");
     static_assert((MPAD == 64 && NT % 8 == 0) || (MPAD == 128 && NT % 16 == 0), "bad MMA N");
     static_assert(NT <= 256 && V % 16 == 0, "bad shape");
     static_assert(RT % CH == 0, "chunking");
@@ -167,7 +180,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
             mbar_init(in_empty(s), C::NWE);
         }
         for (int t = 0; t < C::P; ++t) {
-            mbar_init(bready(t), 4);
+            mbar_init(bready(t), C::WPT);
             mbar_init(accfull(t), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -200,12 +213,14 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
 
     if (warp < C::NWE) {
         // ------------------------------------------------------------ epilogue
-        const int tile = warp >> 2, qd = warp & 3;
+        const int tile = warp / C::WPT, sub = (warp % C::WPT) >> 2, qd = warp & 3;
         const int half = (C::MPAD == 64) ? (lane >> 4) : 0;
         const int j = (C::MPAD == 64) ? qd * 16 + (lane & 15) : qd * 32 + lane;
         const bool jv = j < V;
-        const int nloc = half * C::RT;            // first row within the tile
-        const int row0 = tile * C::R + nloc;      // first state row
+        const int nsub = sub * (C::R / C::SUBS);  // first tile row of this warp
+        const int nloc = nsub + half * C::RT;     // first tile row of this thread
+        const int row0 = tile * C::R + nloc;      // first state row of this thread
+        const int slot = tile * C::SUBS + sub;
         const size_t sbase = (size_t)bh * K * V;
         uint8_t* Bt = smem + C::OFF_B + tile * C::B_BYTES;
 
@@ -222,7 +237,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
         __syncwarp();
         if (lane == 0) mbar_arrive(bready(tile));
 
-        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT);
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT + nsub);
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int c = t / C::TC, tt = t - c * C::TC, s = c % C::S;
@@ -281,7 +296,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 for (int r = 0; r < C::RT; ++r) yp = fmaf(qq[r], h[r], yp);
                 if constexpr (C::MPAD == 64) yp += __shfl_xor_sync(0xffffffffu, yp, 16);
                 if (half == 0 && jv)
-                    reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES)[(tile * C::TC + tt) * V + j] = yp;
+                    reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES)[(slot * C::TC + tt) * V + j] = yp;
             }
             if (p.ckpt != nullptr && jv && (t + 1) < T && ((t + 1) % p.C) == 0) {
                 float* ck = p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * K * V;
@@ -374,8 +389,8 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
             for (int e = lane * 4; e < nt * V; e += 128) {
                 float4 a = *reinterpret_cast<const float4*>(yb + e);
 #pragma unroll
-                for (int tile = 1; tile < C::P; ++tile) {
-                    const float4 b = *reinterpret_cast<const float4*>(yb + tile * C::TC * V + e);
+                for (int sl = 1; sl < C::NSLOT; ++sl) {
+                    const float4 b = *reinterpret_cast<const float4*>(yb + sl * C::TC * V + e);
                     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
                 }
                 *reinterpret_cast<float4*>(yg + e) = a;
