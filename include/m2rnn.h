@@ -93,7 +93,9 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d,
  * (NULL = 0).  ckpt must come from m2rnn_forward with the same inputs and
  * the same dims (including ckpt_stride); the states inside each chunk of C
  * steps are recomputed from it.  Writes dk, dv, dq, df, dW, dH0 (all
- * required, all fp32). */
+ * required, all fp32).  M2RNN_MODE_BF16_TC supports V = 64, K in
+ * {32, 64, 128} and ckpt_stride <= 16 (other shapes return
+ * M2RNN_ERR_UNSUPPORTED_SHAPE); M2RNN_MODE_FP32_DEBUG supports every shape. */
 m2rnn_status m2rnn_backward(const m2rnn_dims* d,
                             const void* k, const void* v, const void* q,
                             const float* f, const void* W, const float* ckpt,

@@ -45,7 +45,7 @@ def lib():
         L.m2rnn_workspace_size.restype = sz
         L.m2rnn_forward.argtypes = [P] + [vp] * 10 + [sz, vp]
         L.m2rnn_forward.restype = i
-        L.m2rnn_backward.argtypes = [P] + [vp] * 14 + [sz, vp]
+        L.m2rnn_backward.argtypes = [P] + [vp] * 15 + [sz, vp]
         L.m2rnn_backward.restype = i
         L.m2rnn_get_device_status.argtypes = [vp, vp]
         L.m2rnn_get_device_status.restype = i

@@ -1,10 +1,531 @@
-// tcgen05 backward (placeholder until the tensor-core BPTT kernel lands).
+// M²RNN backward (BPTT) on the sm_100a tensor cores (tcgen05).
+//
+// For the recurrence of the gist.science technical summary of "M²RNN:
+// Non-Linear RNNs with Matrix-Valued States for Scalable Language Modeling"
+// (§2.1: Z_t = tanh(H_{t-1}W + k_t v_tᵀ), H_t = f_t H_{t-1} + (1-f_t) Z_t)
+// plus the readout y_t = H_tᵀ q_t, with G_t = dL/dH_t (the chain rule of the
+// three equations):
+//   G_t  += q_t dy_tᵀ            dq_t = H_t dy_t
+//   dA_t  = (1 - f_t) G_t ⊙ (1 - Z_t²)
+//   df_t  = <G_t, H_{t-1} - Z_t>  dk_t = dA_t v_t      dv_t = dA_tᵀ k_t
+//   dW   += H_{t-1}ᵀ dA_t         G_{t-1} = f_t G_t + dA_t Wᵀ,   dH0 = G_0.
+// The pages' backward recomputes the states instead of storing them (§2.2);
+// here each chunk of C steps is recomputed from the forward's checkpoint
+// H_{c·C} with exactly the forward kernel's arithmetic (same MMA shapes,
+// same compensated operand, same epilogue), so the states are bit-identical
+// to the forward's.  H_{t-1} and Z_t of the chunk go to a per-CTA workspace
+// scratch (read back only by the thread that wrote them; small enough to
+// stay in L2), then the chunk is walked in reverse.
+//
+// Layout: one CTA per (b, h), the K state rows split into P = 2 tiles with
+// independent chains, the transposed (column) formulation of the forward
+// kernel: TMEM lane j = column j of H / G / dA.  Per reverse step and tile:
+//   G-propagation MMA  D = W · dA_tᵀ   (A = the resident Wᵀ tile read as an
+//                      MN-major operand, B = dA_tᵀ as compensated hi + lo
+//                      bf16, MN-major), so D lane l holds (dA_t Wᵀ)[:, l];
+//   dW MMA             D_W += H_{t-1}ᵀ · dA_t over the tile's rows (both as
+//                      K-major views of the same shared-memory operand
+//                      buffers, hi parts), accumulated in TMEM over all steps.
+// dk and dq reduce over columns: a reduce-scatter across the 16 lanes that
+// share a row block, then a fixed-order sum of the four lane quarters by a
+// storer warp (deterministic).  dv, df and the readout terms are
+// thread-local plus shuffles.  dW partials per (b, h) are summed over the
+// batch by a separate fixed-order reduction kernel.
+//
+// Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace m2rnn {
 
-size_t bwd_tc_workspace(int, int, int, int, int) { return 0; }
+template <int K_>
+struct BwdTcCfg {
+    static constexpr int K = K_, V = 64;
+    static constexpr int P = 2;
+    static constexpr int MPAD = 64;
+    static constexpr int R = K / P;           // rows per tile
+    static constexpr int NT = 2 * R;          // MMA N per tile (hi rows, then lo rows)
+    static constexpr int RT = R / 2;          // rows per epilogue thread
+    static constexpr int CMAX = 16;           // max steps per checkpoint chunk
+    static constexpr int NWE = 4 * P;         // epilogue warps
+    static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
+    static constexpr int NTHREADS = (NWE + 3) * 32;
 
-cudaError_t launch_bwd_tc(const Params&, cudaStream_t) { return cudaErrorNotSupported; }
+    static constexpr int A_BYTES = MPAD * V * 2;
+    static constexpr int B_BYTES = NT * V * 2;
+    static constexpr int ST_K = 0;
+    static constexpr int ST_Q = CMAX * K * 2;
+    static constexpr int ST_V = 2 * CMAX * K * 2;
+    static constexpr int ST_DY = ST_V + CMAX * V * 2;
+    static constexpr int ST_F = ST_DY + CMAX * V * 2;
+    static constexpr int STAGE_BYTES = ((ST_F + CMAX * 4) + 127) / 128 * 128;
+    // partial sums of one chunk
+    static constexpr int DKP = 0;                          // [CMAX][4][K]
+    static constexpr int DQP = DKP + CMAX * 4 * K * 4;     // [CMAX][4][K]
+    static constexpr int DVP = DQP + CMAX * 4 * K * 4;     // [CMAX][P][V]
+    static constexpr int DFP = DVP + CMAX * P * V * 4;     // [CMAX][NWE]
+    static constexpr int PART_BYTES = DFP + CMAX * NWE * 4;
+
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_BS = OFF_A + A_BYTES;         // state operands (recompute; H_{t-1} for dW)
+    static constexpr int OFF_BD = OFF_BS + P * B_BYTES;    // dA operands
+    static constexpr int OFF_RING = OFF_BD + P * B_BYTES;
+    static constexpr int OFF_PART = OFF_RING + 2 * STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
+    static constexpr int NBAR = 4 + 2 * P + 2;
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
+    static constexpr int ACC_COLS = P * NT;                // per-tile accumulators
+    static constexpr int DW_COL = ACC_COLS;                // dW accumulator (V columns)
+    static constexpr int TMEM_COLS = (ACC_COLS + V <= 128) ? 128 : (ACC_COLS + V <= 256) ? 256 : 512;
+
+    static_assert(K == 32 || K == 64 || K == 128, "K");
+    static_assert(R % 16 == 0, "dW MMA needs 16-row k-steps");
+    static_assert(SMEM_BYTES <= 227 * 1024, "smem");
+};
+
+// In-place reduce-scatter of N values over the 16 lanes of a half-warp.
+// Afterwards this lane holds, in v[0 .. N/16) (or v[0] when N <= 16), the
+// sums over the 16 lanes of the values at the indices given by rs16_index.
+template <int N>
+__device__ __forceinline__ void rs16(float (&v)[N], int lane) {
+    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int m = 8 >> k;
+        if (k < L) {
+            const int n = N >> k;
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < N / 2; ++i) {
+                if (i < n / 2) {
+                    const float send = up ? v[i] : v[i + n / 2];
+                    const float keep = up ? v[i + n / 2] : v[i];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < (N >> L); ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], m);
+        }
+    }
+}
+// Index (within the N values) of v[e] after rs16.
+template <int N>
+__device__ __forceinline__ int rs16_index(int lane, int e) {
+    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
+    int idx = e;
+#pragma unroll
+    for (int k = 0; k < L; ++k) idx += (N >> (k + 1)) * ((lane >> (3 - k)) & 1);
+    return idx;
+}
+// Lanes that write the rs16 result (duplicates are skipped when N < 16).
+template <int N>
+__device__ __forceinline__ bool rs16_writer(int lane) {
+    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
+    return (lane & ((1 << (4 - L)) - 1)) == 0;
+}
+
+template <int K>
+__global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(const Params p) {
+    using C = BwdTcCfg<K>;
+    constexpr int V = C::V;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int hd = bh % p.H;
+    const int T = p.T, CS = p.C;
+    const int nck = (T + CS - 1) / CS;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    auto in_full = [&](int s) { return bar(s); };
+    auto in_empty = [&](int s) { return bar(2 + s); };
+    auto bready = [&](int t) { return bar(4 + t); };
+    auto accfull = [&](int t) { return bar(4 + C::P + t); };
+    const uint32_t pfull = bar(4 + 2 * C::P), pempty = bar(5 + 2 * C::P);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* part = reinterpret_cast<float*>(smem + C::OFF_PART);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(in_full(s), 1);
+            mbar_init(in_empty(s), C::NWE);
+        }
+        for (int t = 0; t < C::P; ++t) {
+            mbar_init(bready(t), 4);
+            mbar_init(accfull(t), 1);
+        }
+        mbar_init(pfull, C::NWE);
+        mbar_init(pempty, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    // Wᵀ tile, K-major for the recompute MMA (element (m = j, k = l) = W[l][j]); the
+    // same bytes read as an MN-major operand give A(m = l, k = j) = W[l][j] for the
+    // G-propagation MMA.
+    {
+        const uint16_t* Wg = static_cast<const uint16_t*>(p.W) + (size_t)hd * V * V;
+        for (int idx = threadIdx.x; idx < V * V; idx += C::NTHREADS) {
+            const int l = idx / V, j = idx % V;
+            *reinterpret_cast<uint16_t*>(smem + C::OFF_A + (j >> 3) * (V * 16) + (l >> 3) * 128 + (j & 7) * 16 +
+                                         (l & 7) * 2) = Wg[l * V + j];
+        }
+    }
+    fence_proxy_async_smem();
+    if (warp == C::W_PROD) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < C::NWE) {
+        // ------------------------------------------------------------ epilogue
+        const int tile = warp >> 2, qd = warp & 3;
+        const int half = lane >> 4;
+        const int j = qd * 16 + (lane & 15);
+        const int nloc = half * C::RT;
+        const int row0 = tile * C::R + nloc;
+        const size_t sbase = (size_t)bh * K * V;
+        uint8_t* Bs = smem + C::OFF_BS + tile * C::B_BYTES;
+        uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT);
+        float* Sst = p.scratch + (size_t)bh * (2 * CS + 1) * K * V;   // states H_{c0+u}, u = 0..len
+        float* Sz = Sst + (size_t)(CS + 1) * K * V;                   // Z_{c0+u}, u = 0..len-1
+        auto sidx = [&](int u, int r) { return (size_t)u * K * V + (size_t)(row0 + r) * V + j; };
+
+        float G[C::RT];
+#pragma unroll
+        for (int r = 0; r < C::RT; ++r) G[r] = p.dHT != nullptr ? p.dHT[sbase + (size_t)(row0 + r) * V + j] : 0.f;
+        float fprev = 0.f;
+        uint32_t nacc = 0;
+        bool ok = true;
+        for (int ci = 0; ci < nck && ok; ++ci) {
+            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0), s = ci & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (ci >> 1) & 1, abort_flag, p));
+            if (!ok) break;
+            const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            // ------------------------------------------------ recompute the chunk
+            {
+                float h[C::RT];
+                const float* ck = p.ckpt + ((size_t)bh * nck + c) * K * V;
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) {
+                    h[r] = ck[(size_t)(row0 + r) * V + j];
+                    Sst[sidx(0, r)] = h[r];
+                }
+                write_state_operand<C>(Bs, h, j, nloc);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bready(tile));
+                for (int u = 0; u < len; ++u) {
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
+                    if (!ok) break;
+                    ++nacc;
+                    tc_fence_after();
+                    const float vj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
+                    const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
+                    uint32_t ahi[C::RT], alo[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase, ahi);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, alo);
+                    float kk[C::RT];
+                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
+                    tc_wait_ld();
+                    reg_fence(ahi);
+                    reg_fence(alo);
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r) {
+                        float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
+                        a = fmaf(kk[r], vj, a);
+                        const float z = tanh_exp(a);
+                        h[r] = fmaf(g, z - h[r], h[r]);
+                        Sz[sidx(u, r)] = z;
+                        Sst[sidx(u + 1, r)] = h[r];
+                    }
+                    tc_fence_before();
+                    if (u + 1 < len) {
+                        write_state_operand<C>(Bs, h, j, nloc);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bready(tile));
+                    }
+                }
+                if (!ok) break;
+            }
+            // ------------------------------------------------ reverse over the chunk
+            if (ci >= 1) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(pempty, (ci - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            for (int u = len - 1; u >= 0; --u) {
+                if (u < len - 1) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
+                    if (!ok) break;
+                    ++nacc;
+                    tc_fence_after();
+                    uint32_t dhi[C::RT], dlo[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase, dhi);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, dlo);
+                    tc_wait_ld();
+                    reg_fence(dhi);
+                    reg_fence(dlo);
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r)
+                        G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                    tc_fence_before();
+                }
+                const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_DY + u * V * 2 + j * 2));
+                const float vj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
+                const float ft = *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
+                float qq[C::RT], kk[C::RT];
+                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_Q + u * K * 2) + row0, qq);
+                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
+                float dA[C::RT], Hp[C::RT], pq[C::RT];
+                float dfp = 0.f, dvp = 0.f;
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) {
+                    const float hprev = Sst[sidx(u, r)];
+                    const float hcur = Sst[sidx(u + 1, r)];
+                    const float z = Sz[sidx(u, r)];
+                    G[r] = fmaf(qq[r], dyj, G[r]);
+                    pq[r] = hcur * dyj;
+                    dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
+                    dfp = fmaf(G[r], hprev - z, dfp);
+                    dvp = fmaf(dA[r], kk[r], dvp);
+                    Hp[r] = hprev;
+                }
+                write_state_operand<C, true>(Bd, dA, j, nloc);
+                write_state_operand<C, true>(Bs, Hp, j, nloc);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bready(tile));
+                // reductions (off the critical path)
+                float pk[C::RT];
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) pk[r] = dA[r] * vj;
+                rs16<C::RT>(pk, lane);
+                rs16<C::RT>(pq, lane);
+                if (rs16_writer<C::RT>(lane)) {
+#pragma unroll
+                    for (int e = 0; e < (C::RT >= 16 ? C::RT / 16 : 1); ++e) {
+                        const int row = row0 + rs16_index<C::RT>(lane, e);
+                        part[(C::DKP / 4) + (u * 4 + qd) * K + row] = pk[e];
+                        part[(C::DQP / 4) + (u * 4 + qd) * K + row] = pq[e];
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
+                if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
+                dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
+                if (half == 0) part[(C::DVP / 4) + (u * C::P + tile) * V + j] = dvp;
+                fprev = ft;
+            }
+            if (!ok) break;
+            // G_{c0-1} = f_{c0} G_{c0} + dA_{c0} Wᵀ
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
+            if (!ok) break;
+            ++nacc;
+            tc_fence_after();
+            {
+                uint32_t dhi[C::RT], dlo[C::RT];
+                tmem_ld_16x32bx2<C::RT, C::RT>(tbase, dhi);
+                tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, dlo);
+                tc_wait_ld();
+                reg_fence(dhi);
+                reg_fence(dlo);
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r)
+                    G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(in_empty(s));
+                mbar_arrive(pfull);
+            }
+        }
+        if (ok) {
+#pragma unroll
+            for (int r = 0; r < C::RT; ++r) p.dH0[sbase + (size_t)(row0 + r) * V + j] = G[r];
+        }
+    } else if (warp == C::W_PROD) {
+        // ------------------------------------------------------------ producer (chunks in reverse order)
+        int last = -1;
+        for (int ci = 0; ci < nck; ++ci) {
+            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0), s = ci & 1;
+            if (ci >= 2) {
+                const bool ok =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(in_empty(s), ((ci >> 1) - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            if (lane < len) reinterpret_cast<float*>(st + C::ST_F)[lane] = p.f[(size_t)bh * T + c0 + lane];
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t kb = (uint32_t)(len * K * 2), vb = (uint32_t)(len * V * 2);
+                mbar_arrive_expect_tx(in_full(s), 2 * kb + 2 * vb);
+                const size_t rk = ((size_t)bh * T + c0) * K, rv = ((size_t)bh * T + c0) * V;
+                bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + rk, kb, in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + rk, kb, in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + rv, vb, in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_DY), static_cast<const uint16_t*>(p.dy) + rv, vb, in_full(s));
+            }
+            last = ci;
+        }
+        if (lane == 0)
+            for (int ci = max(0, last - 1); ci <= last; ++ci) mbar_wait_drain(in_full(ci & 1), (ci >> 1) & 1, p);
+        __syncwarp();
+    } else if (warp == C::W_MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t a0 = smem_u32(smem + C::OFF_A);
+            constexpr uint32_t idesc_fwd = idesc_bf16_f32(C::MPAD, C::NT, 0, 1);
+            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MPAD, C::NT, 1, 1);
+            constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
+            uint32_t nbr[C::P];
+            int issued[C::P];
+#pragma unroll
+            for (int i = 0; i < C::P; ++i) {
+                nbr[i] = 0;
+                issued[i] = -1;
+            }
+            bool first_dw = true, ok = true;
+            for (int ci = 0; ci < nck && ok; ++ci) {
+                const int c = nck - 1 - ci, len = min(CS, T - c * CS);
+                for (int u = 0; u < 2 * len && ok; ++u) {
+                    const bool rev = u >= len;
+#pragma unroll
+                    for (int tile = 0; tile < C::P; ++tile) {
+                        if (!mbar_wait_bounded(bready(tile), nbr[tile] & 1, abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
+                        ++nbr[tile];
+                        tc_fence_after();
+                        const uint32_t bs = smem_u32(smem + C::OFF_BS + tile * C::B_BYTES);
+                        const uint32_t bd = smem_u32(smem + C::OFF_BD + tile * C::B_BYTES);
+                        const uint32_t dt = tmem + (uint32_t)(tile * C::NT);
+                        if (!rev) {
+#pragma unroll
+                            for (int ks = 0; ks < V / 16; ++ks)
+                                tc_mma_f16_ss(dt, smem_desc(a0 + ks * 256, 128, V * 16),
+                                              smem_desc(bs + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_fwd,
+                                              ks > 0 ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int ks = 0; ks < V / 16; ++ks)
+                                tc_mma_f16_ss(dt, smem_desc(a0 + ks * 2 * V * 16, V * 16, 128),
+                                              smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
+                                              ks > 0 ? 1u : 0u);
+#pragma unroll
+                            for (int ks = 0; ks < C::R / 16; ++ks) {
+                                tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::NT * 16),
+                                              smem_desc(bd + ks * 256, 128, C::NT * 16), idesc_w,
+                                              (first_dw && ks == 0) ? 0u : 1u);
+                            }
+                            first_dw = false;
+                        }
+                        tc_commit(accfull(tile));
+                        issued[tile] = (int)(nbr[tile] - 1);
+                    }
+                }
+            }
+#pragma unroll
+            for (int tile = 0; tile < C::P; ++tile)
+                if (issued[tile] >= 0) mbar_wait_drain(accfull(tile), (uint32_t)issued[tile] & 1, p);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ partial-sum storer
+        for (int ci = 0; ci < nck; ++ci) {
+            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0);
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull, ci & 1, abort_flag, p));
+            if (!ok) break;
+            for (int e = lane; e < len * K; e += 32) {
+                const int u = e / K, i = e % K;
+                const float* pk = part + C::DKP / 4 + (u * 4) * K + i;
+                const float* pq = part + C::DQP / 4 + (u * 4) * K + i;
+                const size_t o = ((size_t)bh * T + c0 + u) * K + i;
+                p.dk[o] = ((pk[0] + pk[K]) + pk[2 * K]) + pk[3 * K];
+                p.dq[o] = ((pq[0] + pq[K]) + pq[2 * K]) + pq[3 * K];
+            }
+            for (int e = lane; e < len * V; e += 32) {
+                const int u = e / V, jj = e % V;
+                float sv = 0.f;
+#pragma unroll
+                for (int tile = 0; tile < C::P; ++tile) sv += part[C::DVP / 4 + (u * C::P + tile) * V + jj];
+                p.dv[((size_t)bh * T + c0 + u) * V + jj] = sv;
+            }
+            if (lane < len) {
+                float sf = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::NWE; ++w) sf += part[C::DFP / 4 + lane * C::NWE + w];
+                p.df[(size_t)bh * T + c0 + lane] = sf;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pempty);
+        }
+    }
+
+    // dW partial of this (b, h): TMEM lane l (M = 64 layout) holds row l of Σ H_{t-1}ᵀ dA_t
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp < 4 && *abort_flag == 0) {
+        uint32_t w[32];
+        tmem_ld_16x32bx2<32, 32>(tmem + ((uint32_t)(warp * 32) << 16) + C::DW_COL, w);
+        tc_wait_ld();
+        reg_fence(w);
+        const int l = warp * 16 + (lane & 15), j0 = (lane >> 4) * 32;
+        float* dst = p.dW_part + ((size_t)bh * V + l) * V + j0;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(w[e]), __uint_as_float(w[e + 1]),
+                                                             __uint_as_float(w[e + 2]), __uint_as_float(w[e + 3]));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == C::W_PROD) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int K>
+static cudaError_t launch_bwd_tc_k(const Params& p, cudaStream_t stream) {
+    using C = BwdTcCfg<K>;
+    auto kern = m2rnn_bwd_tc_kernel<K>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<p.B * p.H, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_dw_reduce(p, stream);
+}
+
+bool bwd_tc_supported(int K, int V, int C) {
+    return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64>::CMAX;
+}
+
+size_t bwd_tc_workspace(int B, int H, int K, int V, int C) {
+    if (!bwd_tc_supported(K, V, C)) return 0;
+    return sizeof(float) * ((size_t)B * H * V * V + (size_t)B * H * (2 * C + 1) * K * V);
+}
+
+cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s) {
+    if (!bwd_tc_supported(p.K, p.V, p.C)) return cudaErrorNotSupported;
+    switch (p.K) {
+        case 32: return launch_bwd_tc_k<32>(p, s);
+        case 64: return launch_bwd_tc_k<64>(p, s);
+        case 128: return launch_bwd_tc_k<128>(p, s);
+    }
+    return cudaErrorNotSupported;
+}
 
 }  // namespace m2rnn

@@ -42,6 +42,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace m2rnn {
 
@@ -91,66 +92,6 @@ struct FwdTcCfg {
     static_assert(RT % CH == 0, "chunking");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
-
-// Loads n bf16 values (n = 4 or a multiple of 8; 8- or 16-byte aligned) from shared memory.
-template <int N>
-__device__ __forceinline__ void lds_bf16(const uint16_t* src, float (&out)[N]) {
-    if constexpr (N % 8 == 0) {
-#pragma unroll
-        for (int g = 0; g < N / 8; ++g) {
-            const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * g);
-            out[8 * g + 0] = bf16lo_to_f32(w.x); out[8 * g + 1] = bf16hi_to_f32(w.x);
-            out[8 * g + 2] = bf16lo_to_f32(w.y); out[8 * g + 3] = bf16hi_to_f32(w.y);
-            out[8 * g + 4] = bf16lo_to_f32(w.z); out[8 * g + 5] = bf16hi_to_f32(w.z);
-            out[8 * g + 6] = bf16lo_to_f32(w.w); out[8 * g + 7] = bf16hi_to_f32(w.w);
-        }
-    } else {
-        static_assert(N == 4, "lds_bf16");
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        out[0] = bf16lo_to_f32(w.x); out[1] = bf16hi_to_f32(w.x);
-        out[2] = bf16lo_to_f32(w.y); out[3] = bf16hi_to_f32(w.y);
-    }
-}
-
-// hi / lo bf16 pair of two fp32 values, packed two per 32-bit word
-// (element with the lower index in the low half).
-__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
-    hi = __byte_perm(b0, b1, 0x7632);
-    const float l0 = x0 - __uint_as_float(b0 & 0xFFFF0000u);
-    const float l1 = x1 - __uint_as_float(b1 & 0xFFFF0000u);
-    const __nv_bfloat162 lp = __floats2bfloat162_rn(l0, l1);
-    lo = *reinterpret_cast<const uint32_t*>(&lp);
-}
-
-// Writes this thread's RT state values of column j into the MN-major B
-// operand of its tile: element (k = j, n) lives at
-//   (j/8)·(NT·16) + (n/8)·128 + (j%8)·16 + (n%8)·2,
-// hi values at n = nloc + r, lo values at n = R + nloc + r.
-template <class C>
-__device__ __forceinline__ void write_state_operand(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
-    uint8_t* colbase = Bt + (j >> 3) * (C::NT * 16) + (j & 7) * 16;
-    if constexpr (C::RT % 8 == 0) {
-#pragma unroll
-        for (int g = 0; g < C::RT / 8; ++g) {
-            uint4 hi, lo;
-            split_pack(h[8 * g + 0], h[8 * g + 1], hi.x, lo.x);
-            split_pack(h[8 * g + 2], h[8 * g + 3], hi.y, lo.y);
-            split_pack(h[8 * g + 4], h[8 * g + 5], hi.z, lo.z);
-            split_pack(h[8 * g + 6], h[8 * g + 7], hi.w, lo.w);
-            const int n = nloc + 8 * g;
-            *reinterpret_cast<uint4*>(colbase + (n >> 3) * 128) = hi;
-            *reinterpret_cast<uint4*>(colbase + ((C::R + n) >> 3) * 128) = lo;
-        }
-    } else {
-        uint2 hi, lo;
-        split_pack(h[0], h[1], hi.x, lo.x);
-        split_pack(h[2], h[3], hi.y, lo.y);
-        const int n = nloc;
-        *reinterpret_cast<uint2*>(colbase + (n >> 3) * 128 + (n & 7) * 2) = hi;
-        *reinterpret_cast<uint2*>(colbase + ((C::R + n) >> 3) * 128 + ((C::R + n) & 7) * 2) = lo;
-    }
-}
 
 template <int K, int V>
 __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
@@ -261,8 +202,9 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
             for (int c0 = 0; c0 < C::RT; c0 += C::CH) {
                 uint32_t ahi[C::CH], alo[C::CH];
                 if constexpr (C::MPAD == 64) {
-                    tmem_ld_16x32bx2<C::CH, C::CH>(tbase + c0, ahi);
-                    tmem_ld_16x32bx2<C::CH, C::CH>(tbase + C::R + c0, alo);
+                    // the two half-warps own rows [0, RT) and [RT, 2RT) of the warp's block
+                    tmem_ld_16x32bx2<C::CH, C::RT>(tbase + c0, ahi);
+                    tmem_ld_16x32bx2<C::CH, C::RT>(tbase + C::R + c0, alo);
                 } else {
                     tmem_ld_32x32b<C::CH>(tbase + c0, ahi);
                     tmem_ld_32x32b<C::CH>(tbase + C::R + c0, alo);
@@ -276,7 +218,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 for (int r = 0; r < C::CH; ++r) {
                     float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
                     a = fmaf(kk[r], vj, a);
-                    const float z = tanh_approx(a);
+                    const float z = tanh_exp(a);
                     h[c0 + r] = fmaf(g, z - h[c0 + r], h[c0 + r]);
                 }
             }

@@ -17,6 +17,10 @@ cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s);
 // Deterministic dW[h] = sum_b dW_part[b, h] (fixed ascending order).
 cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
 
+// Shapes the tensor-core backward supports (V = 64, K in {32, 64, 128},
+// checkpoint stride <= 16).
+bool bwd_tc_supported(int K, int V, int C);
+
 // Workspace bytes beyond the 256-byte status header.
 size_t bwd_fp32_workspace(int B, int H, int K, int V, int C);
 size_t bwd_tc_workspace(int B, int H, int K, int V, int C);

@@ -90,6 +90,8 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     if ((seq && (!k || !v || !q || !f || !dy || !dk || !dv || !dq || !df || !ckpt)) || (d->H > 0 && (!W || !dW)) ||
         (state && !dH0) || !workspace)
         return M2RNN_ERR_INVALID_ARG;
+    if (d->mode == M2RNN_MODE_BF16_TC && !m2rnn::bwd_tc_supported(d->K, d->V, d->ckpt_stride))
+        return M2RNN_ERR_UNSUPPORTED_SHAPE;
     const void* ptrs[] = {k, v, q, f, W, ckpt, dy, dHT, dk, dv, dq, df, dW, dH0, workspace};
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return M2RNN_ERR_MISALIGNED;

@@ -158,42 +158,31 @@ __device__ __forceinline__ void tmem_ld_32x32b<32>(uint32_t taddr, uint32_t (&r)
 }
 
 template <int N, int SPLIT>
-__device__ __forceinline__ void tmem_ld_16x32bx2(uint32_t taddr, uint32_t (&r)[N]);
-#define M2RNN_LD16_4(S)                                                                              \
-    template <>                                                                                      \
-    __device__ __forceinline__ void tmem_ld_16x32bx2<4, S>(uint32_t taddr, uint32_t(&r)[4]) {        \
-        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0,%1,%2,%3}, [%4], " #S ";"           \
-                     : M2RNN_R4(r)                                                                   \
-                     : "r"(taddr));                                                                  \
+__device__ __forceinline__ void tmem_ld_16x32bx2(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 4 || N == 8 || N == 16 || N == 32, "tmem_ld_16x32bx2 width");
+    if constexpr (N == 4) {
+        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0,%1,%2,%3}, [%4], %5;"
+                     : M2RNN_R4(r)
+                     : "r"(taddr), "n"(SPLIT));
+    } else if constexpr (N == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;"
+                     : M2RNN_R8(r)
+                     : "r"(taddr), "n"(SPLIT));
+    } else if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;"
+            : M2RNN_R8o(r, 0), M2RNN_R8o(r, 8)
+            : "r"(taddr), "n"(SPLIT));
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+            : M2RNN_R8o(r, 0), M2RNN_R8o(r, 8), M2RNN_R8o(r, 16), M2RNN_R8o(r, 24)
+            : "r"(taddr), "n"(SPLIT));
     }
-#define M2RNN_LD16_8(S)                                                                              \
-    template <>                                                                                      \
-    __device__ __forceinline__ void tmem_ld_16x32bx2<8, S>(uint32_t taddr, uint32_t(&r)[8]) {        \
-        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], " #S ";" \
-                     : M2RNN_R8(r)                                                                   \
-                     : "r"(taddr));                                                                  \
-    }
-#define M2RNN_LD16_16(S)                                                                             \
-    template <>                                                                                      \
-    __device__ __forceinline__ void tmem_ld_16x32bx2<16, S>(uint32_t taddr, uint32_t(&r)[16]) {      \
-        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "                                     \
-                     "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], " #S ";"        \
-                     : M2RNN_R8o(r, 0), M2RNN_R8o(r, 8)                                              \
-                     : "r"(taddr));                                                                  \
-    }
-#define M2RNN_LD16_32(S)                                                                             \
-    template <>                                                                                      \
-    __device__ __forceinline__ void tmem_ld_16x32bx2<32, S>(uint32_t taddr, uint32_t(&r)[32]) {      \
-        asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "                                     \
-                     "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                       \
-                     "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], " #S ";" \
-                     : M2RNN_R8o(r, 0), M2RNN_R8o(r, 8), M2RNN_R8o(r, 16), M2RNN_R8o(r, 24)          \
-                     : "r"(taddr));                                                                  \
-    }
-M2RNN_LD16_4(4)
-M2RNN_LD16_8(8)
-M2RNN_LD16_16(16)
-M2RNN_LD16_32(32)
+}
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, no swizzle ("interleaved" canonical layout
@@ -226,6 +215,15 @@ __device__ __forceinline__ float tanh_approx(float x) {
     float y;
     asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+// tanh from the identity tanh(x) = 1 - 2 / (1 + e^{2x}), evaluated with the
+// exponential and fast-division intrinsics (two SFU operations).  Absolute
+// error below ~1e-6 on the whole line (saturates to +-1 for large |x|), about
+// three orders of magnitude below tanh.approx.f32, whose ~2^-11 relative error
+// the backward's sensitivity over long sequences would amplify.
+__device__ __forceinline__ float tanh_exp(float x) {
+    const float e = __expf(2.f * x);
+    return 1.f - __fdividef(2.f, 1.f + e);
 }
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

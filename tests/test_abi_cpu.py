@@ -86,3 +86,15 @@ def test_backward_argument_errors(L):
 
 def test_status_query_rejects_null(L):
     assert L.m2rnn_get_device_status(None, None) == _lib.ERR_INVALID_ARG
+
+
+def test_binding_signatures_match_header(L):
+    """Each ctypes declaration has exactly the parameter count of the header prototype
+    (a missing parameter shifts every later argument, e.g. the stream handle)."""
+    header = open(os.path.join(ROOT, "include", "m2rnn.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    for name in _lib.EXPORTS:
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", header)
+        assert m, name
+        params = [x for x in m.group(1).split(",") if x.strip() and x.strip() != "void"]
+        assert len(getattr(L, name).argtypes) == len(params), (name, len(params))

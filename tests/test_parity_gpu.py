@@ -183,3 +183,85 @@ def test_full_size_forward_sampled(name):
     ys = torch.stack([y[b, h] for b, h in pairs])[None]
     HTs = torch.stack([HT[b, h] for b, h in pairs])[None]
     _check_fwd("full_" + name, ys, HTs, yr, HTr, "bf16")
+
+
+# ---------------------------------------------------------------- backward
+
+
+def _oracle_bwd(x, dHT=None):
+    return oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], dHT)
+
+
+def _gpu_fwd_bwd(xc, C, dHT=None):
+    a = api()
+    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True)
+    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], dHT, ckpt_stride=C)
+    torch.cuda.synchronize()
+    assert a.device_status() == 0
+    return g
+
+
+def _check_grads(name, g, gr, tol):
+    errs = {}
+    for n in ("dk", "dv", "dq", "df", "dW", "dH0"):
+        ref = gr[n]
+        if np.linalg.norm(ref) == 0:
+            errs[n] = float(np.abs(g[n].double().cpu().numpy()).max())
+            continue
+        _, errs[n] = _errs(g[n], ref)
+    _log(name, **{n + "_rel": e for n, e in errs.items()})
+    for n, e in errs.items():
+        assert e <= tol, (n, e, errs)
+
+
+@pytest.mark.parametrize("K", [32, 64, 128])
+@pytest.mark.parametrize("T,C", [(1, 16), (5, 4), (17, 8), (40, 16), (33, 5)])
+@pytest.mark.parametrize("with_dHT", [False, True])
+def test_tc_backward_small(K, T, C, with_dHT):
+    w = Workload("bw", B=2, H=3, T=T, K=K, V=64, h0_range=0.5, backward=True, seed=K + T + C)
+    x = make_inputs(w)
+    dHT = torch.randn(2, 3, K, 64, generator=torch.Generator().manual_seed(7)) if with_dHT else None
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, C, None if dHT is None else dHT.cuda())
+    gr = _oracle_bwd(x, dHT)
+    _check_grads("tc_bwd_K%d_T%d_C%d_dHT%d" % (K, T, C, int(with_dHT)), g, gr, GRAD_REL)
+
+
+@pytest.mark.parametrize("K,V", [(16, 16), (32, 64), (64, 64), (64, 128), (128, 32)])
+@pytest.mark.parametrize("T,C", [(1, 3), (19, 4), (40, 16)])
+def test_fp32_backward_small(K, V, T, C):
+    w = Workload("bwd", B=2, H=2, T=T, K=K, V=V, mode="fp32", h0_range=0.5, backward=True, seed=K + V + T)
+    x = make_inputs(w)
+    dHT = torch.randn(2, 2, K, V, generator=torch.Generator().manual_seed(3))
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, C, dHT.cuda())
+    gr = _oracle_bwd(x, dHT)
+    _check_grads("fp32_bwd_K%d_V%d_T%d_C%d" % (K, V, T, C), g, gr, 1e-4)
+
+
+def test_tc_backward_unsupported_shape():
+    from non_linear_matrix_persistent_b200._lib import ERR_UNSUPPORTED_SHAPE, M2RNNError
+    w = Workload("u", B=1, H=1, T=4, K=64, V=128, backward=True)
+    xc = _cuda(make_inputs(w))
+    _, _, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=4, want_ckpt=True)
+    with pytest.raises(M2RNNError) as e:
+        api().backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=4)
+    assert e.value.status == ERR_UNSUPPORTED_SHAPE
+
+
+def test_train_workload_sampled_head():
+    """Full-size training workload (fwd with checkpoints + BPTT) in the launch
+    configuration the benchmark times; the oracle checks one whole head (all
+    batch rows, so dW[h] is complete) plus the bound on every output."""
+    w = WORKLOADS["layer410m_train"]
+    x = make_inputs(w)
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, 16)
+    for n, t in g.items():
+        assert torch.isfinite(t).all(), n
+    h = 5
+    sel = {n: (None if t is None else t[:, h:h + 1].contiguous()) for n, t in x.items() if n != "W"}
+    sel["W"] = x["W"][h:h + 1].contiguous()
+    gr = _oracle_bwd(sel)
+    gs = {n: (t[:, h:h + 1] if n != "dW" else t[h:h + 1]) for n, t in g.items()}
+    _check_grads("full_layer410m_train_head%d" % h, gs, gr, GRAD_REL)
