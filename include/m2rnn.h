@@ -104,6 +104,27 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d,
                             float* dW, float* dH0,
                             void* workspace, size_t ws_bytes, m2rnn_stream_t stream);
 
+/* Allocation-free m2rnn_backward (the pages describe no such variant: it is
+ * an interface addition of this library).  For callers that cannot allocate
+ * device memory when they need gradients, e.g. code running under CUDA-graph
+ * capture or services that forbid allocator calls after start-up.  Same
+ * arguments and results as m2rnn_backward minus the workspace: the scratch
+ * comes from a 32 MiB array compiled into the library, which every GPU that
+ * loads the library keeps until the process exits.
+ *  - Problems with m2rnn_workspace_size(d, 1) > 32 MiB return
+ *    M2RNN_ERR_WORKSPACE and launch nothing.
+ *  - All calls share the array: calls whose kernels overlap on the GPU race
+ *    and give wrong results; order them on one stream.
+ *  - The first call on a device looks up the array's device address (no
+ *    allocation); make it before any stream capture starts.
+ *  - Device-side wait timeouts are not reported by this entry point. */
+m2rnn_status m2rnn_backward_noalloc(const m2rnn_dims* d,
+                                    const void* k, const void* v, const void* q,
+                                    const float* f, const void* W, const float* ckpt,
+                                    const void* dy, const float* dHT,
+                                    float* dk, float* dv, float* dq, float* df,
+                                    float* dW, float* dH0, m2rnn_stream_t stream);
+
 /* Synchronises `stream`, reads and clears the status word in `workspace`.
  * Returns M2RNN_OK or M2RNN_ERR_DEVICE_TIMEOUT (or M2RNN_ERR_CUDA). */
 m2rnn_status m2rnn_get_device_status(void* workspace, m2rnn_stream_t stream);

@@ -16,8 +16,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_C
 MODE_BF16_TC, MODE_FP32_DEBUG = 0, 1
 
 # Every entry point declared in include/m2rnn.h.
-EXPORTS = ("m2rnn_workspace_size", "m2rnn_forward", "m2rnn_backward", "m2rnn_get_device_status",
-           "m2rnn_status_string", "m2rnn_set_wait_limit_ns")
+EXPORTS = ("m2rnn_workspace_size", "m2rnn_forward", "m2rnn_backward", "m2rnn_backward_noalloc",
+           "m2rnn_get_device_status", "m2rnn_status_string", "m2rnn_set_wait_limit_ns")
 
 
 class Dims(ctypes.Structure):
@@ -47,6 +47,8 @@ def lib():
         L.m2rnn_forward.restype = i
         L.m2rnn_backward.argtypes = [P] + [vp] * 15 + [sz, vp]
         L.m2rnn_backward.restype = i
+        L.m2rnn_backward_noalloc.argtypes = [P] + [vp] * 14 + [vp]
+        L.m2rnn_backward_noalloc.restype = i
         L.m2rnn_get_device_status.argtypes = [vp, vp]
         L.m2rnn_get_device_status.restype = i
         L.m2rnn_status_string.argtypes = [i]
