@@ -48,9 +48,15 @@ struct BwdTcCfg {
     static constexpr int MPAD = 64;
     static constexpr int R = K / P;           // rows per tile
     static constexpr int NT = 2 * R;          // MMA N per tile (hi rows, then lo rows)
-    static constexpr int RT = R / 2;          // rows per epilogue thread
+    // two warps per TMEM lane quarter and tile (each owning half of the tile's
+    // rows) when the tile is large enough: the reverse step is issue-bound, and
+    // more warps with fewer rows each raise the issue rate
+    static constexpr int SUBS = (R / 4 >= 4) ? 2 : 1;
+    static constexpr int WPT = 4 * SUBS;      // epilogue warps per tile
+    static constexpr int RT = R / (2 * SUBS); // rows per epilogue thread
     static constexpr int CMAX = 16;           // max steps per checkpoint chunk
-    static constexpr int NWE = 4 * P;         // epilogue warps
+    static constexpr int NWE = P * WPT;       // epilogue warps
+    static constexpr int NSLOT = P * SUBS;    // dv partials per (t, j)
     static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
     static constexpr int NTHREADS = (NWE + 3) * 32;
 
@@ -65,8 +71,8 @@ struct BwdTcCfg {
     // partial sums of one chunk
     static constexpr int DKP = 0;                          // [CMAX][4][K]
     static constexpr int DQP = DKP + CMAX * 4 * K * 4;     // [CMAX][4][K]
-    static constexpr int DVP = DQP + CMAX * 4 * K * 4;     // [CMAX][P][V]
-    static constexpr int DFP = DVP + CMAX * P * V * 4;     // [CMAX][NWE]
+    static constexpr int DVP = DQP + CMAX * 4 * K * 4;     // [CMAX][NSLOT][V]
+    static constexpr int DFP = DVP + CMAX * NSLOT * V * 4; // [CMAX][NWE]
     static constexpr int PART_BYTES = DFP + CMAX * NWE * 4;
 
     static constexpr int OFF_A = 0;
@@ -83,6 +89,8 @@ struct BwdTcCfg {
 
     static_assert(K == 32 || K == 64 || K == 128, "K");
     static_assert(R % 16 == 0, "dW MMA needs 16-row k-steps");
+    static_assert(RT % 4 == 0 && NWE * 32 * RT == K * V, "row split");
+    static_assert(NTHREADS <= 1024, "block size");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
 
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
             mbar_init(in_empty(s), C::NWE);
         }
         for (int t = 0; t < C::P; ++t) {
-            mbar_init(bready(t), 4);
+            mbar_init(bready(t), C::WPT);
             mbar_init(accfull(t), 1);
         }
         mbar_init(pfull, C::NWE);
@@ -187,18 +195,36 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
 
     if (warp < C::NWE) {
         // ------------------------------------------------------------ epilogue
-        const int tile = warp >> 2, qd = warp & 3;
+        const int tile = warp / C::WPT, sub = (warp % C::WPT) >> 2, qd = warp & 3;
         const int half = lane >> 4;
         const int j = qd * 16 + (lane & 15);
-        const int nloc = half * C::RT;
+        const int nsub = sub * (C::R / C::SUBS);   // first tile row of this warp
+        const int nloc = nsub + half * C::RT;      // first tile row of this thread
         const int row0 = tile * C::R + nloc;
+        const int slot = tile * C::SUBS + sub;
         const size_t sbase = (size_t)bh * K * V;
         uint8_t* Bs = smem + C::OFF_BS + tile * C::B_BYTES;
         uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
-        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT);
+        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT + nsub);
+        // Scratch, thread-contiguous: step u, thread t holds its RT values at
+        // u·K·V + t·RT (16-byte vector accesses, each warp touching one
+        // contiguous block).  Only the thread that wrote a value reads it back.
         float* Sst = p.scratch + (size_t)bh * (2 * CS + 1) * K * V;   // states H_{c0+u}, u = 0..len
         float* Sz = Sst + (size_t)(CS + 1) * K * V;                   // Z_{c0+u}, u = 0..len-1
-        auto sidx = [&](int u, int r) { return (size_t)u * K * V + (size_t)(row0 + r) * V + j; };
+        const size_t tslot = (size_t)threadIdx.x * C::RT;
+        auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
+            float4* d = reinterpret_cast<float4*>(base + (size_t)u * K * V + tslot);
+#pragma unroll
+            for (int g = 0; g < C::RT / 4; ++g) d[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        };
+        auto ld_vec = [&](const float* base, int u, float (&v)[C::RT]) {
+            const float4* s4 = reinterpret_cast<const float4*>(base + (size_t)u * K * V + tslot);
+#pragma unroll
+            for (int g = 0; g < C::RT / 4; ++g) {
+                const float4 x = s4[g];
+                v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
+            }
+        };
 
         float G[C::RT];
 #pragma unroll
@@ -216,10 +242,8 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 float h[C::RT];
                 const float* ck = p.ckpt + ((size_t)bh * nck + c) * K * V;
 #pragma unroll
-                for (int r = 0; r < C::RT; ++r) {
-                    h[r] = ck[(size_t)(row0 + r) * V + j];
-                    Sst[sidx(0, r)] = h[r];
-                }
+                for (int r = 0; r < C::RT; ++r) h[r] = ck[(size_t)(row0 + r) * V + j];
+                st_vec(Sst, 0, h);
                 write_state_operand<C>(Bs, h, j, nloc);
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -239,15 +263,16 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                     tc_wait_ld();
                     reg_fence(ahi);
                     reg_fence(alo);
+                    float zz[C::RT];
 #pragma unroll
                     for (int r = 0; r < C::RT; ++r) {
                         float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
                         a = fmaf(kk[r], vj, a);
-                        const float z = tanh_exp(a);
-                        h[r] = fmaf(g, z - h[r], h[r]);
-                        Sz[sidx(u, r)] = z;
-                        Sst[sidx(u + 1, r)] = h[r];
+                        zz[r] = tanh_exp(a);
+                        h[r] = fmaf(g, zz[r] - h[r], h[r]);
                     }
+                    st_vec(Sz, u, zz);
+                    st_vec(Sst, u + 1, h);
                     tc_fence_before();
                     if (u + 1 < len) {
                         write_state_operand<C>(Bs, h, j, nloc);
@@ -263,6 +288,14 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(pempty, (ci - 1) & 1, abort_flag, p));
                 if (!ok) break;
             }
+            // scratch values of the step being processed: H_{t-1}, H_t and Z_t.  The
+            // next step's Z and H_{t-1} are loaded right after each step's arrive, so
+            // their L2 latency overlaps the MMA round trip (H_t of the next step is
+            // this step's H_{t-1}).
+            float zc[C::RT], hpc[C::RT], hcc[C::RT];
+            ld_vec(Sz, len - 1, zc);
+            ld_vec(Sst, len - 1, hpc);
+            ld_vec(Sst, len, hcc);
             for (int u = len - 1; u >= 0; --u) {
                 if (u < len - 1) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
                     ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
@@ -286,25 +319,28 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 float qq[C::RT], kk[C::RT];
                 lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_Q + u * K * 2) + row0, qq);
                 lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
-                float dA[C::RT], Hp[C::RT], pq[C::RT];
+                float dA[C::RT], pq[C::RT];
                 float dfp = 0.f, dvp = 0.f;
 #pragma unroll
                 for (int r = 0; r < C::RT; ++r) {
-                    const float hprev = Sst[sidx(u, r)];
-                    const float hcur = Sst[sidx(u + 1, r)];
-                    const float z = Sz[sidx(u, r)];
+                    const float z = zc[r];
                     G[r] = fmaf(qq[r], dyj, G[r]);
-                    pq[r] = hcur * dyj;
+                    pq[r] = hcc[r] * dyj;
                     dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
-                    dfp = fmaf(G[r], hprev - z, dfp);
+                    dfp = fmaf(G[r], hpc[r] - z, dfp);
                     dvp = fmaf(dA[r], kk[r], dvp);
-                    Hp[r] = hprev;
                 }
                 write_state_operand<C, true>(Bd, dA, j, nloc);
-                write_state_operand<C, true>(Bs, Hp, j, nloc);
+                write_state_operand<C, true>(Bs, hpc, j, nloc);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready(tile));
+                if (u > 0) {
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r) hcc[r] = hpc[r];
+                    ld_vec(Sz, u - 1, zc);
+                    ld_vec(Sst, u - 1, hpc);
+                }
                 // reductions (off the critical path)
                 float pk[C::RT];
 #pragma unroll
@@ -323,7 +359,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
                 if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
                 dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
-                if (half == 0) part[(C::DVP / 4) + (u * C::P + tile) * V + j] = dvp;
+                if (half == 0) part[(C::DVP / 4) + (u * C::NSLOT + slot) * V + j] = dvp;
                 fprev = ft;
             }
             if (!ok) break;
@@ -459,7 +495,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 const int u = e / V, jj = e % V;
                 float sv = 0.f;
 #pragma unroll
-                for (int tile = 0; tile < C::P; ++tile) sv += part[C::DVP / 4 + (u * C::P + tile) * V + jj];
+                for (int sl = 0; sl < C::NSLOT; ++sl) sv += part[C::DVP / 4 + (u * C::NSLOT + sl) * V + jj];
                 p.dv[((size_t)bh * T + c0 + u) * V + jj] = sv;
             }
             if (lane < len) {
