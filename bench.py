@@ -8,20 +8,21 @@ workloads.  Prints ONE JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own shard of the
-global batch (weak scaling; the ranks' inputs differ by seed).  The only
-exchange is the all-reduce of dW (the gradient of the shared per-head W is a
-sum over the global batch) in training workloads.
+global batch (weak scaling; same W, rank-seeded data).  The only exchange is
+the all-reduce of dW (the gradient of the shared per-head W is a sum over the
+global batch) in training workloads.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on the host
 cores on a bounded sample of the same workload (whole (b, h) pairs at full
-length), because there is no runnable reference implementation.
+length), because the pages describe no runnable reference implementation.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
-import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -34,12 +35,16 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from non_linear_matrix_persistent_b200 import WORKLOADS, make_inputs  # noqa: E402
+from non_linear_matrix_persistent_b200.inputs import make_shard_inputs  # noqa: E402
 
 METRIC = "M2RNN layer fwd(+bwd) tokens/s on 1 B200"
 DEFAULT_WORKLOAD = "layer410m_train"
+CKPT_STRIDE = 16
 L2_FLUSH_BYTES = 256 << 20
-MUFU_PER_SM_PER_CLK = 16      # tanh.approx results per SM per clock (4 per SM sub-partition)
 NUM_SMS = 148
+SFU_PER_SM_PER_CLK = 16      # special-function (exp / reciprocal) results per SM per clock
+SFU_PER_TANH = 2             # tanh = 1 - 2/(1 + e^{2x}): one exp and one reciprocal
+CSRC = os.path.join(ROOT, "non_linear_matrix_persistent_b200", "csrc")
 
 
 def _peaks():
@@ -52,16 +57,15 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.gpu, self.period = gpu_index, period_ms
+        self.proc = self.path = None
 
     def __enter__(self):
         try:
@@ -69,14 +73,16 @@ class ClockSampler:
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period)],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)   # let the first sample land before the timed region
         except Exception:
             self.proc = None
         return self
 
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -96,59 +102,89 @@ class ClockSampler:
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             for n, v in zip(names, r[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][2]),
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
-def algorithmic_counts(w):
-    """Per-launch algorithmic work of the forward scan (the dominant kernel)."""
-    steps = w.B * w.H * w.T
-    return {
-        "tanh": steps * w.K * w.V,                          # one tanh per state element per step
-        "gemm_flop": 2.0 * steps * w.K * w.V * w.V,          # H_{t-1}W
-        "hbm_bytes": steps * ((2 * w.K + w.V) * 2 + 4 + 4 * w.V),  # k,q,v (bf16), f, y (fp32)
-    }
+def per_step_counts(w):
+    """Algorithmic work per (b, h, t) of each kernel (stated in the design doc §6)."""
+    K, V, C = w.K, w.V, CKPT_STRIDE
+    fwd = {"tanh": K * V, "flop": 2.0 * K * V * V,
+           "bytes": (2 * K + V) * 2 + 4 + 4 * V + (4.0 * K * V / C if w.backward else 0.0)}
+    bwd = {"tanh": K * V, "flop": 3 * 2.0 * K * V * V,
+           "bytes": (2 * K + 2 * V) * 2 + 4 + (2 * K + V) * 4 + 4 + 4.0 * K * V / C}
+    return fwd, bwd
+
+
+def measured_traffic(kernel_file: str, profile_md: str):
+    """DRAM bytes per launch recorded in a profiles/ summary, when that summary
+    was taken from the current kernel source (sha256 of the .cu file); else None."""
+    try:
+        src = open(os.path.join(CSRC, kernel_file), "rb").read()
+        text = open(os.path.join(ROOT, "profiles", profile_md)).read()
+    except OSError:
+        return None
+    digest = hashlib.sha256(src).hexdigest()[:16]
+    m = re.search(r"source sha256\[:16\] of %s: `([0-9a-f]+)`" % re.escape(kernel_file), text)
+    t = re.search(r"DRAM traffic per launch: ([0-9.]+) bytes", text)
+    if m and t and m.group(1) == digest:
+        return float(t.group(1))
+    return None
+
+
+def _sample_pairs(w, cores, budget_flop):
+    pairs_total = w.B * w.H
+    per_pair = 2.0 * w.T * w.K * w.V * w.V * (4.0 if w.backward else 1.0)
+    npairs = int(max(1, min(pairs_total, cores, budget_flop // per_pair)))
+    return [(i % w.B, (i * 7) % w.H) for i in range(npairs)]
+
+
+def _oracle_sample(w, pairs, cores):
+    from oracle import oracle
+    x = make_inputs(w)
+
+    def sel(n):
+        return torch.stack([x[n][b, h] for b, h in pairs])[None]
+    W = torch.stack([x["W"][h] for _, h in pairs])
+    H0 = None if x["H0"] is None else sel("H0")
+    args = (sel("k"), sel("v"), sel("q"), sel("f"), W, H0)
+
+    def run():
+        if w.backward:
+            oracle.backward(*args, sel("dY"), nthreads=cores)
+        else:
+            oracle.forward(*args, nthreads=cores)
+    return run
 
 
 def run_reference(args, w):
     """fp64 CPU oracle on a bounded sample of (b, h) pairs at full length."""
     from oracle import oracle
     cores = oracle.default_threads()
-    pairs_total = w.B * w.H
-    # sample size: enough pairs to keep every core busy, bounded by the work budget
-    per_pair_flop = 2.0 * w.T * w.K * w.V * w.V * (4.0 if w.backward else 1.0)
-    budget = float(os.environ.get("M2RNN_REF_FLOP_BUDGET", 2.0e10))
-    npairs = int(max(1, min(pairs_total, cores, budget // per_pair_flop)))
-    x = make_inputs(w)
-    pairs = [(i % w.B, (i * 7) % w.H) for i in range(npairs)]
-
-    def sel(n):
-        return torch.stack([x[n][b, h] for b, h in pairs])[None]
-    k, v, q, f = sel("k"), sel("v"), sel("q"), sel("f")
-    W = torch.stack([x["W"][h] for _, h in pairs])
-    H0 = None if x["H0"] is None else sel("H0")
-    dY = sel("dY") if w.backward else None
+    pairs = _sample_pairs(w, cores, float(os.environ.get("M2RNN_REF_FLOP_BUDGET", 2.0e10)))
+    run = _oracle_sample(w, pairs, cores)
     times = []
     for it in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        if w.backward:
-            oracle.backward(k, v, q, f, W, H0, dY, nthreads=cores)
-        else:
-            oracle.forward(k, v, q, f, W, H0, nthreads=cores)
-        dt = time.perf_counter() - t0
+        run()
         if it >= args.warmup:
-            times.append(dt)
-    tok = w.B * w.T * npairs / pairs_total
+            times.append(time.perf_counter() - t0)
+    tok = w.B * w.T * len(pairs) / (w.B * w.H)
     value = tok * len(times) / sum(times)
-    sample = "%d of %d (b,h) pairs at full T=%d, %s" % (npairs, pairs_total, w.T,
+    sample = "%d of %d (b,h) pairs at full T=%d, %s" % (len(pairs), w.B * w.H, w.T,
                                                          "fwd+bwd" if w.backward else "fwd")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
@@ -161,32 +197,21 @@ def run_reference(args, w):
 def cpu_baseline(w):
     from oracle import oracle
     cores = oracle.default_threads()
-    pairs_total = w.B * w.H
-    per_pair_flop = 2.0 * w.T * w.K * w.V * w.V * (4.0 if w.backward else 1.0)
-    npairs = int(max(1, min(pairs_total, cores, 2.0e10 // per_pair_flop)))
-    x = make_inputs(w)
-    pairs = [(i % w.B, (i * 7) % w.H) for i in range(npairs)]
-
-    def sel(n):
-        return torch.stack([x[n][b, h] for b, h in pairs])[None]
-    W = torch.stack([x["W"][h] for _, h in pairs])
-    H0 = None if x["H0"] is None else sel("H0")
+    pairs = _sample_pairs(w, cores, 2.0e10)
+    run = _oracle_sample(w, pairs, cores)
     t0 = time.perf_counter()
-    if w.backward:
-        oracle.backward(sel("k"), sel("v"), sel("q"), sel("f"), W, H0, sel("dY"), nthreads=cores)
-    else:
-        oracle.forward(sel("k"), sel("v"), sel("q"), sel("f"), W, H0, nthreads=cores)
+    run()
     dt = time.perf_counter() - t0
-    tok = w.B * w.T * npairs / pairs_total
+    tok = w.B * w.T * len(pairs) / (w.B * w.H)
     return {"value": tok / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": "%d of %d (b,h) pairs at full T=%d, %s, one run" % (
-                npairs, pairs_total, w.T, "fwd+bwd" if w.backward else "fwd")}
+                len(pairs), w.B * w.H, w.T, "fwd+bwd" if w.backward else "fwd")}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -194,8 +219,8 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    from non_linear_matrix_persistent_b200 import parallel
+    rank, world = parallel.world_from_env()
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
 
@@ -206,32 +231,31 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    dist = None
     if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        parallel.init("nccl", timeout_s=120)
 
     from non_linear_matrix_persistent_b200 import api
-    wr = w.with_(seed=w.seed + rank)
-    x_host = make_inputs(wr)
+    x_host = make_shard_inputs(w, rank)
     x = {n: (None if t is None else t.to(dev)) for n, t in x_host.items()}
-    C = 16
+    C = CKPT_STRIDE
     B, H, T, K, V = w.B, w.H, w.T, w.K, w.V
     outs = {"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev),
             "ckpt": torch.empty(B, H, (T + C - 1) // C, K, V, device=dev)}
     gouts = {}
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        y, HT, ck = api.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=C,
-                                want_ckpt=w.backward, out=outs)
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=C, want_ckpt=w.backward, out=outs)
+        if ev is not None:
+            ev[1].record(stream)
         if w.backward:
-            g = api.backward(x["k"], x["v"], x["q"], x["f"], x["W"], ck, x["dY"], ckpt_stride=C, out=gouts)
+            g = api.backward(x["k"], x["v"], x["q"], x["f"], x["W"], outs["ckpt"], x["dY"], ckpt_stride=C, out=gouts)
             gouts.update(g)
-            if dist is not None:
-                dist.all_reduce(g["dW"])
-        return y
+            parallel.allreduce_dW(g["dW"])
+        if ev is not None:
+            ev[2].record(stream)
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(args.warmup):
@@ -240,45 +264,29 @@ def main():
     if api.device_status(dev) != 0:
         raise RuntimeError("device-side wait ran out during warm-up")
 
-    # kernel-only timing: per-step CUDA events on the launching stream, L2 flushed between steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if dist is not None:
+    # kernel timing: per-step CUDA events on the launching stream, L2 flushed between steps
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.zero_()
-            ev[i][0].record(stream)
-            fwd_ev[i][0].record(stream)
-            api.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=C, want_ckpt=w.backward,
-                        out=outs)
-            fwd_ev[i][1].record(stream)
-            if w.backward:
-                g = api.backward(x["k"], x["v"], x["q"], x["f"], x["W"], outs["ckpt"], x["dY"], ckpt_stride=C,
-                                 out=gouts)
-                gouts.update(g)
-                if dist is not None:
-                    dist.all_reduce(g["dW"])
-            ev[i][1].record(stream)
+            step(evs[i])
         torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    fwd_ms = [a.elapsed_time(b) for a, b in fwd_ev]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    step_ms = [a.elapsed_time(c) for a, b, c in evs]
+    fwd_ms = [a.elapsed_time(b) for a, b, c in evs]
+    bwd_ms = [b.elapsed_time(c) for a, b, c in evs]
+    total_ms = parallel.max_over_ranks(sum(step_ms), dev)
     if api.device_status(dev) != 0:
         raise RuntimeError("device-side wait ran out during the timed region")
     ms_per_step = total_ms / args.steps
     tokens_per_step = B * T * world
     value = tokens_per_step / (ms_per_step / 1e3)
 
-    # end-to-end through the public API with host buffers: pinned H2D of the
-    # step's inputs, the step, D2H of its results
+    # end to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, the step, D2H of its results (y and, for training, the gradients)
     pinned = {n: (None if t is None else t.pin_memory()) for n, t in x_host.items()}
     res_names = ["y"] + (["dk", "dv", "dq", "df", "dW", "dH0"] if w.backward else [])
     h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
@@ -295,8 +303,7 @@ def main():
         res = {"y": y}
         if w.backward:
             res.update(api.backward(xd["k"], xd["v"], xd["q"], xd["f"], xd["W"], ck, xd["dY"], ckpt_stride=C))
-            if dist is not None:
-                dist.all_reduce(res["dW"])
+            parallel.allreduce_dW(res["dW"])
         for n in res_names:
             if n not in host_out:
                 host_out[n] = torch.empty(res[n].shape, dtype=res[n].dtype, pin_memory=True)
@@ -306,33 +313,41 @@ def main():
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_total = sum(e2e_ms)
-    if dist is not None:
-        t = torch.tensor([e2e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = parallel.max_over_ranks(sum(e2e_ms), dev)
     e2e_value = tokens_per_step / (e2e_total / args.steps / 1e3)
 
     peaks, peak_kind = _peaks()
     clocks = clk.summary()
-    cnt = algorithmic_counts(w)
-    fwd_avg_s = sum(fwd_ms) / len(fwd_ms) / 1e3
-    sm_mhz_peak = float(peaks.get("sm_max_mhz", 1965.0))
-    mufu_peak = NUM_SMS * MUFU_PER_SM_PER_CLK * sm_mhz_peak * 1e6 / 1e9   # Gtanh/s
-    achieved_tanh = cnt["tanh"] / fwd_avg_s / 1e9
-    roofline = {"kernel": "m2rnn_fwd_tc_kernel", "bound": "alu", "unit": "Gtanh/s",
-                "achieved": achieved_tanh, "peak": mufu_peak, "frac": achieved_tanh / mufu_peak,
-                "peak_source": "derived: %d SMs x %d MUFU tanh/clk x %.0f MHz" % (NUM_SMS, MUFU_PER_SM_PER_CLK,
-                                                                                  sm_mhz_peak),
-                "traffic": None,
-                "tensor": {"achieved_tflops": cnt["gemm_flop"] / fwd_avg_s / 1e12,
-                           "peak_tflops": peaks["bf16_tflops"],
-                           "frac": cnt["gemm_flop"] / fwd_avg_s / 1e12 / peaks["bf16_tflops"],
-                           "peak_kind": peak_kind},
-                "hbm": {"achieved_gbs": cnt["hbm_bytes"] / fwd_avg_s / 1e9, "peak_gbs": peaks["hbm_gbs"],
-                        "frac": cnt["hbm_bytes"] / fwd_avg_s / 1e9 / peaks["hbm_gbs"], "peak_kind": peak_kind},
-                "fwd_ms": fwd_avg_s * 1e3,
-                "cycles_per_step": fwd_avg_s * sm_mhz_peak * 1e6 / T}
+    sm_mhz = clocks.get("sm_mhz") or float(peaks.get("sm_max_mhz", 1965.0))
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    cf, cb = per_step_counts(w)
+    units = B * H * T   # (b, h, t) steps per launch on this rank
+    kernels = {}
+    for name, ms_list, cnt, src, prof in (
+            ("m2rnn_fwd_tc_kernel", fwd_ms, cf, "fwd_tc.cu", "m2rnn_fwd_tc_layer410m_train.md"),
+            ("m2rnn_bwd_tc_kernel", bwd_ms, cb, "bwd_tc.cu", "m2rnn_bwd_tc_layer410m_train.md")):
+        if name.startswith("m2rnn_bwd") and not w.backward:
+            continue
+        s = statistics.mean(ms_list) / 1e3
+        sfu = SFU_PER_TANH * cnt["tanh"] * units / s / 1e9
+        sfu_peak = NUM_SMS * SFU_PER_SM_PER_CLK * sm_max * 1e6 / 1e9
+        traffic = measured_traffic(src, prof) if w.name == "layer410m_train" else None
+        kernels[name] = {
+            "ms": s * 1e3,
+            "bound": "alu", "unit": "GSFUop/s", "achieved": sfu, "peak": sfu_peak, "frac": sfu / sfu_peak,
+            "peak_source": "derived: %d SMs x %d SFU results/clk x %.0f MHz; %d SFU ops per tanh" % (
+                NUM_SMS, SFU_PER_SM_PER_CLK, sm_max, SFU_PER_TANH),
+            "traffic": traffic,
+            "algorithmic_per_step": cnt,
+            "tensor": {"achieved_tflops": cnt["flop"] * units / s / 1e12, "peak_tflops": peaks["bf16_tflops"],
+                       "frac": cnt["flop"] * units / s / 1e12 / peaks["bf16_tflops"], "peak_kind": peak_kind},
+            "hbm": {"achieved_gbs": cnt["bytes"] * units / s / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                    "frac": cnt["bytes"] * units / s / 1e9 / peaks["hbm_gbs"], "peak_kind": peak_kind},
+            "cycles_per_recurrence_step": s * sm_mhz * 1e6 / T,
+        }
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    roofline = dict(kernel=dom, **{k: v for k, v in kernels[dom].items()})
+    roofline["kernels"] = kernels
     launches = args.steps * (1 + (2 if w.backward else 0))
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -347,7 +362,9 @@ def main():
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if dist is not None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
         dist.destroy_process_group()
 
 

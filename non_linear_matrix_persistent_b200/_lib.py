@@ -17,7 +17,8 @@ MODE_BF16_TC, MODE_FP32_DEBUG = 0, 1
 
 # Every entry point declared in include/m2rnn.h.
 EXPORTS = ("m2rnn_workspace_size", "m2rnn_forward", "m2rnn_backward", "m2rnn_backward_noalloc",
-           "m2rnn_get_device_status", "m2rnn_status_string", "m2rnn_set_wait_limit_ns")
+           "m2rnn_get_device_status", "m2rnn_status_string", "m2rnn_set_wait_limit_ns",
+           "m2rnn_debug_set_fault")
 
 
 class Dims(ctypes.Structure):
@@ -55,6 +56,8 @@ def lib():
         L.m2rnn_status_string.restype = ctypes.c_char_p
         L.m2rnn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
         L.m2rnn_set_wait_limit_ns.restype = None
+        L.m2rnn_debug_set_fault.argtypes = [i]
+        L.m2rnn_debug_set_fault.restype = i
         _lib = L
     return _lib
 

@@ -38,6 +38,7 @@ struct Params {
     float* scratch;     // per-CTA recompute scratch (workspace)
     uint32_t* status;   // device status word (workspace)
     uint64_t wait_limit_ns;
+    int fault;          // injected fault (m2rnn_debug_set_fault), 0 = none
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA-wide

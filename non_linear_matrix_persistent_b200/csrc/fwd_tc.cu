@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
         int last = -1;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % C::S;
+            if (p.fault == 1 && c >= 1) break;   // injected: stop feeding the ring after the first chunk
             if (c >= C::S) {
                 const bool ok =
                     __all_sync(0xffffffffu, mbar_wait_bounded(in_empty(s), ((c / C::S) - 1) & 1, abort_flag, p));

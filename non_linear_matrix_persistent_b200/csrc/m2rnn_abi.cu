@@ -11,6 +11,7 @@
 namespace {
 
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_fault{0};
 constexpr size_t kStatusBytes = 256;
 
 bool shape_ok(int n) { return n == 16 || n == 32 || n == 64 || n == 128; }
@@ -30,6 +31,7 @@ m2rnn::Params base_params(const m2rnn_dims* d, void* ws) {
     p.B = d->B; p.H = d->H; p.T = d->T; p.K = d->K; p.V = d->V; p.C = d->ckpt_stride;
     p.status = static_cast<uint32_t*>(ws);
     p.wait_limit_ns = g_wait_limit_ns.load();
+    p.fault = g_fault.load();
     return p;
 }
 
@@ -149,5 +151,11 @@ const char* m2rnn_status_string(m2rnn_status s) {
 }
 
 void m2rnn_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns < 100000ull ? 100000ull : ns); }
+
+int m2rnn_debug_set_fault(int fault) {
+    if (fault != 0 && fault != 1) return M2RNN_ERR_INVALID_ARG;
+    g_fault.store(fault);
+    return M2RNN_OK;
+}
 
 }  // extern "C"

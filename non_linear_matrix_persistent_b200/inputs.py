@@ -95,3 +95,18 @@ def make_inputs(w: Workload, device: Optional[str] = None) -> Dict[str, torch.Te
     if device is not None:
         out = {n: (None if t is None else t.to(device)) for n, t in out.items()}
     return out
+
+
+def make_shard_inputs(w: Workload, rank: int, device: Optional[str] = None) -> Dict[str, torch.Tensor]:
+    """Inputs of data-parallel shard `rank` of a global batch of world·B rows.
+
+    The data (k, v, q, f, H0, dY) of shard r are drawn with seed w.seed + r; the
+    per-head parameter W is the same on every shard (drawn with w.seed), as a
+    shared layer parameter must be.
+    """
+    x = make_inputs(dataclasses.replace(w, seed=w.seed + rank))
+    if rank != 0:
+        x["W"] = make_inputs(w)["W"]
+    if device is not None:
+        x = {n: (None if t is None else t.to(device)) for n, t in x.items()}
+    return x
