@@ -11,26 +11,29 @@
 //   dW   += H_{t-1}ᵀ dA_t         G_{t-1} = f_t G_t + dA_t Wᵀ,   dH0 = G_0.
 // The pages' backward recomputes the states instead of storing them (§2.2);
 // here each chunk of C steps is recomputed from the forward's checkpoint
-// H_{c·C} with exactly the forward kernel's arithmetic (same MMA shapes,
-// same compensated operand, same epilogue), so the states are bit-identical
-// to the forward's.  H_{t-1} and Z_t of the chunk go to a per-CTA workspace
-// scratch (read back only by the thread that wrote them; small enough to
-// stay in L2), then the chunk is walked in reverse.
+// H_{c·C} with exactly the forward kernel's arithmetic (same compensated
+// operand, same epilogue), so the states are bit-identical to the forward's.
+// H_{t-1} and Z_t of the chunk go to a per-CTA workspace scratch (read back
+// only by the thread that wrote them), then the chunk is walked in reverse.
 //
 // Layout: one CTA per (b, h), the K state rows split into P = 2 tiles with
 // independent chains, the transposed (column) formulation of the forward
-// kernel: TMEM lane j = column j of H / G / dA.  Per reverse step and tile:
-//   G-propagation MMA  D = W · dA_tᵀ   (A = the resident Wᵀ tile read as an
-//                      MN-major operand, B = dA_tᵀ as compensated hi + lo
-//                      bf16, MN-major), so D lane l holds (dA_t Wᵀ)[:, l];
-//   dW MMA             D_W += H_{t-1}ᵀ · dA_t over the tile's rows (both as
-//                      K-major views of the same shared-memory operand
-//                      buffers, hi parts), accumulated in TMEM over all steps.
-// dk and dq reduce over columns: a reduce-scatter across the 16 lanes that
-// share a row block, then a fixed-order sum of the four lane quarters by a
-// storer warp (deterministic).  dv, df and the readout terms are
-// thread-local plus shuffles.  dW partials per (b, h) are summed over the
-// batch by a separate fixed-order reduction kernel.
+// kernel: the epilogue thread that owns column j of H also owns column j of
+// G and dA.  Per step and tile:
+//   recompute MMA      D = Ã_f · H_{t-1}ᵀ,  Ã_f = Wᵀ plus the row dy_{t-1}
+//   G-propagation MMA  D = Ã_g · dA_tᵀ,     Ã_g = W  plus the row v_t
+//   dW MMA             D_W += H_{t-1}ᵀ · dA_t (M = 64), accumulated in TMEM
+// The first two are M = 128 MMAs: rows 32q + r (r < 16) of Ã hold row
+// 16q + r of Wᵀ / W, so TMEM lane 32q + r is column 16q + r exactly as in the
+// M = 64 layout the forward uses, and the spare row 16 carries one extra
+// vector.  D lane 16 therefore holds the two column reductions that would
+// otherwise take cross-lane shuffles:
+//   recompute:      Σ_l dy_{t-1}[l] H_{t-1}[i, l] = dq_{t-1}[i]
+//   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
+// dv, df are thread-local plus shuffles; their per-warp partials are summed
+// in a fixed order by a storer warp, and the dW partials per (b, h) are
+// summed over the batch in a fixed order by a separate kernel, so results
+// are deterministic.
 //
 // Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16.
 #include <cuda_bf16.h>
@@ -45,7 +48,9 @@ template <int K_>
 struct BwdTcCfg {
     static constexpr int K = K_, V = 64;
     static constexpr int P = 2;
-    static constexpr int MPAD = 64;
+    static constexpr int MPAD = 64;           // M of the dW MMA and of the state-operand layout
+    static constexpr int MX = 128;            // M of the recompute and G-propagation MMAs
+    static constexpr int XLANE = 16;          // TMEM lane (and Ã row) of the extra output
     static constexpr int R = K / P;           // rows per tile
     static constexpr int NT = 2 * R;          // MMA N per tile (hi rows, then lo rows)
     // two warps per TMEM lane quarter and tile (each owning half of the tile's
@@ -60,23 +65,21 @@ struct BwdTcCfg {
     static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
     static constexpr int NTHREADS = (NWE + 3) * 32;
 
-    static constexpr int A_BYTES = MPAD * V * 2;
+    static constexpr int AX_BYTES = MX * V * 2;            // one extended A operand
     static constexpr int B_BYTES = NT * V * 2;
     static constexpr int ST_K = 0;
     static constexpr int ST_Q = CMAX * K * 2;
     static constexpr int ST_V = 2 * CMAX * K * 2;
-    static constexpr int ST_DY = ST_V + CMAX * V * 2;
-    static constexpr int ST_F = ST_DY + CMAX * V * 2;
+    static constexpr int ST_DY = ST_V + CMAX * V * 2;      // CMAX + 1 rows: row r is step c0 - 1 + r
+    static constexpr int ST_F = ST_DY + (CMAX + 1) * V * 2;
     static constexpr int STAGE_BYTES = ((ST_F + CMAX * 4) + 127) / 128 * 128;
-    // partial sums of one chunk
-    static constexpr int DKP = 0;                          // [CMAX][4][K]
-    static constexpr int DQP = DKP + CMAX * 4 * K * 4;     // [CMAX][4][K]
-    static constexpr int DVP = DQP + CMAX * 4 * K * 4;     // [CMAX][NSLOT][V]
+    static constexpr int DVP = 0;                          // [CMAX][NSLOT][V]
     static constexpr int DFP = DVP + CMAX * NSLOT * V * 4; // [CMAX][NWE]
     static constexpr int PART_BYTES = DFP + CMAX * NWE * 4;
 
-    static constexpr int OFF_A = 0;
-    static constexpr int OFF_BS = OFF_A + A_BYTES;         // state operands (recompute; H_{t-1} for dW)
+    static constexpr int OFF_AF = 0;                       // Ã_f per tile (K-major)
+    static constexpr int OFF_AG = OFF_AF + P * AX_BYTES;   // Ã_g per tile (MN-major)
+    static constexpr int OFF_BS = OFF_AG + P * AX_BYTES;   // state operands (recompute; H_{t-1} for dW)
     static constexpr int OFF_BD = OFF_BS + P * B_BYTES;    // dA operands
     static constexpr int OFF_RING = OFF_BD + P * B_BYTES;
     static constexpr int OFF_PART = OFF_RING + 2 * STAGE_BYTES;
@@ -89,51 +92,47 @@ struct BwdTcCfg {
 
     static_assert(K == 32 || K == 64 || K == 128, "K");
     static_assert(R % 16 == 0, "dW MMA needs 16-row k-steps");
+    static_assert(NT % 16 == 0 && NT <= 256, "N of an M = 128 MMA");
     static_assert(RT % 4 == 0 && NWE * 32 * RT == K * V, "row split");
     static_assert(NTHREADS <= 1024, "block size");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
 
-// In-place reduce-scatter of N values over the 16 lanes of a half-warp.
-// Afterwards this lane holds, in v[0 .. N/16) (or v[0] when N <= 16), the
-// sums over the 16 lanes of the values at the indices given by rs16_index.
-template <int N>
-__device__ __forceinline__ void rs16(float (&v)[N], int lane) {
-    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
+// Row of an extended A operand that carries state column x (lanes 32q + r, r < 16).
+__device__ __forceinline__ int xrow(int x) { return 32 * (x >> 4) + (x & 15); }
+// Byte offset of element (m, k) in a K-major extended A operand (V values of k).
+__device__ __forceinline__ int af_off(int m, int k) {
+    return (m >> 3) * (64 * 16) + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
+}
+// Byte offset of element (m, k) in an MN-major extended A operand (128 values of m).
+__device__ __forceinline__ int ag_off(int m, int k) {
+    return (k >> 3) * (128 * 16) + (m >> 3) * 128 + (k & 7) * 16 + (m & 7) * 2;
+}
+
+// Stores the extra output row (TMEM lane XLANE) of one tile, hi + lo parts
+// of its R columns summed, to dst[0 .. R).  Warp-collective over lane quarter
+// 0; thread XLANE stores, and only when `store` is set.
+template <class C>
+__device__ __forceinline__ void store_xrow(uint32_t tcol, float* dst, bool store) {
+    constexpr int CHK = C::R < 16 ? C::R : 16;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int m = 8 >> k;
-        if (k < L) {
-            const int n = N >> k;
-            const bool up = (lane & m) != 0;
+    for (int c0 = 0; c0 < C::R; c0 += CHK) {
+        uint32_t hi[CHK], lo[CHK];
+        tmem_ld_32x32b<CHK>(tcol + c0, hi);
+        tmem_ld_32x32b<CHK>(tcol + C::R + c0, lo);
+        tc_wait_ld();
+        reg_fence(hi);
+        reg_fence(lo);
+        if (store) {
+            float4* d = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
-            for (int i = 0; i < N / 2; ++i) {
-                if (i < n / 2) {
-                    const float send = up ? v[i] : v[i + n / 2];
-                    const float keep = up ? v[i + n / 2] : v[i];
-                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < (N >> L); ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], m);
+            for (int g = 0; g < CHK / 4; ++g)
+                d[g] = make_float4(__uint_as_float(hi[4 * g]) + __uint_as_float(lo[4 * g]),
+                                   __uint_as_float(hi[4 * g + 1]) + __uint_as_float(lo[4 * g + 1]),
+                                   __uint_as_float(hi[4 * g + 2]) + __uint_as_float(lo[4 * g + 2]),
+                                   __uint_as_float(hi[4 * g + 3]) + __uint_as_float(lo[4 * g + 3]));
         }
     }
-}
-// Index (within the N values) of v[e] after rs16.
-template <int N>
-__device__ __forceinline__ int rs16_index(int lane, int e) {
-    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
-    int idx = e;
-#pragma unroll
-    for (int k = 0; k < L; ++k) idx += (N >> (k + 1)) * ((lane >> (3 - k)) & 1);
-    return idx;
-}
-// Lanes that write the rs16 result (duplicates are skipped when N < 16).
-template <int N>
-__device__ __forceinline__ bool rs16_writer(int lane) {
-    constexpr int L = N >= 16 ? 4 : (N == 8 ? 3 : (N == 4 ? 2 : (N == 2 ? 1 : 0)));
-    return (lane & ((1 << (4 - L)) - 1)) == 0;
 }
 
 template <int K>
@@ -172,15 +171,22 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    // Wᵀ tile, K-major for the recompute MMA (element (m = j, k = l) = W[l][j]); the
-    // same bytes read as an MN-major operand give A(m = l, k = j) = W[l][j] for the
-    // G-propagation MMA.
+    // Extended A operands of both tiles: zero everything, then W into the
+    // permuted rows (the extra row is written per step by the epilogue).
+    for (int i = threadIdx.x; i < 2 * C::P * C::AX_BYTES / 16; i += C::NTHREADS)
+        reinterpret_cast<uint4*>(smem + C::OFF_AF)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
     {
         const uint16_t* Wg = static_cast<const uint16_t*>(p.W) + (size_t)hd * V * V;
         for (int idx = threadIdx.x; idx < V * V; idx += C::NTHREADS) {
             const int l = idx / V, j = idx % V;
-            *reinterpret_cast<uint16_t*>(smem + C::OFF_A + (j >> 3) * (V * 16) + (l >> 3) * 128 + (j & 7) * 16 +
-                                         (l & 7) * 2) = Wg[l * V + j];
+            const uint16_t w = Wg[l * V + j];
+#pragma unroll
+            for (int t = 0; t < C::P; ++t) {
+                // Ã_f(m, k = l) = Wᵀ[j][l] at m = xrow(j);  Ã_g(m, k = j) = W[l][j] at m = xrow(l)
+                *reinterpret_cast<uint16_t*>(smem + C::OFF_AF + t * C::AX_BYTES + af_off(xrow(j), l)) = w;
+                *reinterpret_cast<uint16_t*>(smem + C::OFF_AG + t * C::AX_BYTES + ag_off(xrow(l), j)) = w;
+            }
         }
     }
     fence_proxy_async_smem();
@@ -202,9 +208,14 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         const int nloc = nsub + half * C::RT;      // first tile row of this thread
         const int row0 = tile * C::R + nloc;
         const int slot = tile * C::SUBS + sub;
+        const bool xwriter = sub == 0 && half == 0;      // writes element j of the extra A rows
+        const bool xreader = sub == 0 && qd == 0;        // warp that reads TMEM lane XLANE
         const size_t sbase = (size_t)bh * K * V;
         uint8_t* Bs = smem + C::OFF_BS + tile * C::B_BYTES;
         uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
+        uint16_t* xf = reinterpret_cast<uint16_t*>(smem + C::OFF_AF + tile * C::AX_BYTES + af_off(C::XLANE, j));
+        uint16_t* xg = reinterpret_cast<uint16_t*>(smem + C::OFF_AG + tile * C::AX_BYTES + ag_off(C::XLANE, j));
+        const uint32_t tcol = tmem + (uint32_t)(tile * C::NT);
         const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT + nsub);
         // Scratch, thread-contiguous: step u, thread t holds its RT values at
         // u·K·V + t·RT (16-byte vector accesses, each warp touching one
@@ -225,6 +236,11 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
             }
         };
+        // Row t of dq or dk for this tile's rows, from TMEM lane XLANE (reader
+        // warp only; nothing is stored for t < 0).
+        auto emit_xrow = [&](float* out, int t) {
+            store_xrow<C>(tcol, out + ((size_t)bh * T + max(t, 0)) * K + tile * C::R, lane == C::XLANE && t >= 0);
+        };
 
         float G[C::RT];
 #pragma unroll
@@ -234,9 +250,13 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         bool ok = true;
         for (int ci = 0; ci < nck && ok; ++ci) {
             const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0), s = ci & 1;
+            // the chunk holding step T-1 runs one more recompute MMA, for dq_{T-1} = H_{T-1} dy_{T-1}
+            const int nmma = len + (ci == 0 ? 1 : 0);
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (ci >> 1) & 1, abort_flag, p));
             if (!ok) break;
             const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            // dy of step c0 + u, for u = -1 .. len-1 (row -1 only when c0 > 0)
+            auto dy_row = [&](int u) { return reinterpret_cast<const uint16_t*>(st + C::ST_DY + (u + 1) * V * 2); };
             // ------------------------------------------------ recompute the chunk
             {
                 float h[C::RT];
@@ -245,37 +265,43 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 for (int r = 0; r < C::RT; ++r) h[r] = ck[(size_t)(row0 + r) * V + j];
                 st_vec(Sst, 0, h);
                 write_state_operand<C>(Bs, h, j, nloc);
+                if (xwriter) *xf = c0 > 0 ? dy_row(-1)[j] : (uint16_t)0;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready(tile));
-                for (int u = 0; u < len; ++u) {
+                for (int u = 0; u < nmma; ++u) {
                     ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
                     if (!ok) break;
                     ++nacc;
                     tc_fence_after();
-                    const float vj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
-                    const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
-                    uint32_t ahi[C::RT], alo[C::RT];
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase, ahi);
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, alo);
-                    float kk[C::RT];
-                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
-                    tc_wait_ld();
-                    reg_fence(ahi);
-                    reg_fence(alo);
-                    float zz[C::RT];
+                    if (xreader) emit_xrow(p.dq, c0 + u - 1);
+                    if (u < len) {
+                        const float vj =
+                            bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
+                        const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
+                        uint32_t ahi[C::RT], alo[C::RT];
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tbase, ahi);
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, alo);
+                        float kk[C::RT];
+                        lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
+                        tc_wait_ld();
+                        reg_fence(ahi);
+                        reg_fence(alo);
+                        float zz[C::RT];
 #pragma unroll
-                    for (int r = 0; r < C::RT; ++r) {
-                        float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
-                        a = fmaf(kk[r], vj, a);
-                        zz[r] = tanh_exp(a);
-                        h[r] = fmaf(g, zz[r] - h[r], h[r]);
+                        for (int r = 0; r < C::RT; ++r) {
+                            float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
+                            a = fmaf(kk[r], vj, a);
+                            zz[r] = tanh_exp(a);
+                            h[r] = fmaf(g, zz[r] - h[r], h[r]);
+                        }
+                        st_vec(Sz, u, zz);
+                        st_vec(Sst, u + 1, h);
                     }
-                    st_vec(Sz, u, zz);
-                    st_vec(Sst, u + 1, h);
                     tc_fence_before();
-                    if (u + 1 < len) {
+                    if (u + 1 < nmma) {
                         write_state_operand<C>(Bs, h, j, nloc);
+                        if (xwriter) *xf = dy_row(u)[j];
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bready(tile));
@@ -288,16 +314,14 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(pempty, (ci - 1) & 1, abort_flag, p));
                 if (!ok) break;
             }
-            // scratch values of the step being processed: H_{t-1}, H_t and Z_t.  The
-            // next step's Z and H_{t-1} are loaded right after each step's arrive, so
-            // their L2 latency overlaps the MMA round trip (H_t of the next step is
-            // this step's H_{t-1}).
-            float zc[C::RT], hpc[C::RT], hcc[C::RT];
+            // scratch values of the step being processed: H_{t-1} and Z_t.  The
+            // next step's are loaded right after each step's arrive, so their L2
+            // latency overlaps the MMA round trip.
+            float zc[C::RT], hpc[C::RT];
             ld_vec(Sz, len - 1, zc);
             ld_vec(Sst, len - 1, hpc);
-            ld_vec(Sst, len, hcc);
             for (int u = len - 1; u >= 0; --u) {
-                if (u < len - 1) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
+                if (u < len - 1) {   // fold in dA_{t+1} Wᵀ from the previous reverse step; emit dk_{t+1}
                     ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
                     if (!ok) break;
                     ++nacc;
@@ -311,49 +335,34 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
 #pragma unroll
                     for (int r = 0; r < C::RT; ++r)
                         G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                    if (xreader) emit_xrow(p.dk, c0 + u + 1);
                     tc_fence_before();
                 }
-                const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_DY + u * V * 2 + j * 2));
-                const float vj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
+                const float dyj = bf16lo_to_f32(dy_row(u)[j]);
+                const uint16_t vbits = *reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2);
                 const float ft = *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
                 float qq[C::RT], kk[C::RT];
                 lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_Q + u * K * 2) + row0, qq);
                 lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
-                float dA[C::RT], pq[C::RT];
+                float dA[C::RT];
                 float dfp = 0.f, dvp = 0.f;
 #pragma unroll
                 for (int r = 0; r < C::RT; ++r) {
                     const float z = zc[r];
                     G[r] = fmaf(qq[r], dyj, G[r]);
-                    pq[r] = hcc[r] * dyj;
                     dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
                     dfp = fmaf(G[r], hpc[r] - z, dfp);
                     dvp = fmaf(dA[r], kk[r], dvp);
                 }
                 write_state_operand<C, true>(Bd, dA, j, nloc);
                 write_state_operand<C, true>(Bs, hpc, j, nloc);
+                if (xwriter) *xg = vbits;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready(tile));
                 if (u > 0) {
-#pragma unroll
-                    for (int r = 0; r < C::RT; ++r) hcc[r] = hpc[r];
                     ld_vec(Sz, u - 1, zc);
                     ld_vec(Sst, u - 1, hpc);
-                }
-                // reductions (off the critical path)
-                float pk[C::RT];
-#pragma unroll
-                for (int r = 0; r < C::RT; ++r) pk[r] = dA[r] * vj;
-                rs16<C::RT>(pk, lane);
-                rs16<C::RT>(pq, lane);
-                if (rs16_writer<C::RT>(lane)) {
-#pragma unroll
-                    for (int e = 0; e < (C::RT >= 16 ? C::RT / 16 : 1); ++e) {
-                        const int row = row0 + rs16_index<C::RT>(lane, e);
-                        part[(C::DKP / 4) + (u * 4 + qd) * K + row] = pk[e];
-                        part[(C::DQP / 4) + (u * 4 + qd) * K + row] = pq[e];
-                    }
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
@@ -363,7 +372,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 fprev = ft;
             }
             if (!ok) break;
-            // G_{c0-1} = f_{c0} G_{c0} + dA_{c0} Wᵀ
+            // G_{c0-1} = f_{c0} G_{c0} + dA_{c0} Wᵀ; emit dk_{c0}
             ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
             if (!ok) break;
             ++nacc;
@@ -379,6 +388,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 for (int r = 0; r < C::RT; ++r)
                     G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
             }
+            if (xreader) emit_xrow(p.dk, c0);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -405,12 +415,18 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
             __syncwarp();
             if (lane == 0) {
                 const uint32_t kb = (uint32_t)(len * K * 2), vb = (uint32_t)(len * V * 2);
-                mbar_arrive_expect_tx(in_full(s), 2 * kb + 2 * vb);
+                // dy rows c0-1 .. c0+len-1; the row of step c0-1 exists only when c0 > 0
+                const uint32_t dyb = (uint32_t)((len + (c0 > 0 ? 1 : 0)) * V * 2);
+                mbar_arrive_expect_tx(in_full(s), 2 * kb + vb + dyb);
                 const size_t rk = ((size_t)bh * T + c0) * K, rv = ((size_t)bh * T + c0) * V;
+                const uint16_t* dyg = static_cast<const uint16_t*>(p.dy) + rv;
                 bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + rk, kb, in_full(s));
                 bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + rk, kb, in_full(s));
                 bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + rv, vb, in_full(s));
-                bulk_g2s(smem_u32(st + C::ST_DY), static_cast<const uint16_t*>(p.dy) + rv, vb, in_full(s));
+                if (c0 > 0)
+                    bulk_g2s(smem_u32(st + C::ST_DY), dyg - V, dyb, in_full(s));
+                else
+                    bulk_g2s(smem_u32(st + C::ST_DY + V * 2), dyg, dyb, in_full(s));
             }
             last = ci;
         }
@@ -420,9 +436,8 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
     } else if (warp == C::W_MMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t a0 = smem_u32(smem + C::OFF_A);
-            constexpr uint32_t idesc_fwd = idesc_bf16_f32(C::MPAD, C::NT, 0, 1);
-            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MPAD, C::NT, 1, 1);
+            constexpr uint32_t idesc_f = idesc_bf16_f32(C::MX, C::NT, 0, 1);
+            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::NT, 1, 1);
             constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
             uint32_t nbr[C::P];
             int issued[C::P];
@@ -434,8 +449,9 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
             bool first_dw = true, ok = true;
             for (int ci = 0; ci < nck && ok; ++ci) {
                 const int c = nck - 1 - ci, len = min(CS, T - c * CS);
-                for (int u = 0; u < 2 * len && ok; ++u) {
-                    const bool rev = u >= len;
+                const int nmma = len + (ci == 0 ? 1 : 0);
+                for (int u = 0; u < nmma + len && ok; ++u) {
+                    const bool rev = u >= nmma;
 #pragma unroll
                     for (int tile = 0; tile < C::P; ++tile) {
                         if (!mbar_wait_bounded(bready(tile), nbr[tile] & 1, abort_flag, p)) {
@@ -444,19 +460,21 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                         }
                         ++nbr[tile];
                         tc_fence_after();
+                        const uint32_t af = smem_u32(smem + C::OFF_AF + tile * C::AX_BYTES);
+                        const uint32_t ag = smem_u32(smem + C::OFF_AG + tile * C::AX_BYTES);
                         const uint32_t bs = smem_u32(smem + C::OFF_BS + tile * C::B_BYTES);
                         const uint32_t bd = smem_u32(smem + C::OFF_BD + tile * C::B_BYTES);
                         const uint32_t dt = tmem + (uint32_t)(tile * C::NT);
                         if (!rev) {
 #pragma unroll
                             for (int ks = 0; ks < V / 16; ++ks)
-                                tc_mma_f16_ss(dt, smem_desc(a0 + ks * 256, 128, V * 16),
-                                              smem_desc(bs + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_fwd,
+                                tc_mma_f16_ss(dt, smem_desc(af + ks * 256, 128, V * 16),
+                                              smem_desc(bs + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_f,
                                               ks > 0 ? 1u : 0u);
                         } else {
 #pragma unroll
                             for (int ks = 0; ks < V / 16; ++ks)
-                                tc_mma_f16_ss(dt, smem_desc(a0 + ks * 2 * V * 16, V * 16, 128),
+                                tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
                                               smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
                                               ks > 0 ? 1u : 0u);
 #pragma unroll
@@ -478,19 +496,11 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ partial-sum storer
+        // ------------------------------------------------------------ dv / df storer
         for (int ci = 0; ci < nck; ++ci) {
             const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0);
             const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull, ci & 1, abort_flag, p));
             if (!ok) break;
-            for (int e = lane; e < len * K; e += 32) {
-                const int u = e / K, i = e % K;
-                const float* pk = part + C::DKP / 4 + (u * 4) * K + i;
-                const float* pq = part + C::DQP / 4 + (u * 4) * K + i;
-                const size_t o = ((size_t)bh * T + c0 + u) * K + i;
-                p.dk[o] = ((pk[0] + pk[K]) + pk[2 * K]) + pk[3 * K];
-                p.dq[o] = ((pq[0] + pq[K]) + pq[2 * K]) + pq[3 * K];
-            }
             for (int e = lane; e < len * V; e += 32) {
                 const int u = e / V, jj = e % V;
                 float sv = 0.f;
