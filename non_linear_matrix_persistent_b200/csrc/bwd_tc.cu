@@ -16,10 +16,11 @@
 // H_{t-1} and Z_t of the chunk go to a per-CTA workspace scratch (read back
 // only by the thread that wrote them), then the chunk is walked in reverse.
 //
-// Layout: one CTA per (b, h), the K state rows split into P = 2 tiles with
-// independent chains, the transposed (column) formulation of the forward
-// kernel: the epilogue thread that owns column j of H also owns column j of
-// G and dA.  Per step and tile:
+// Layout: one CTA per (b, h) and slice of at most 64 state rows (rows of H
+// evolve independently given W, v_t and f_t), the slice's rows split into
+// P = 2 tiles with independent chains, the transposed (column) formulation
+// of the forward kernel: the epilogue thread that owns column j of H also
+// owns column j of G and dA.  Per step and tile:
 //   recompute MMA      D = Ã_f · H_{t-1}ᵀ,  Ã_f = Wᵀ plus the row dy_{t-1}
 //   G-propagation MMA  D = Ã_g · dA_tᵀ,     Ã_g = W  plus the row v_t
 //   dW MMA             D_W += H_{t-1}ᵀ · dA_t (M = 64), accumulated in TMEM
@@ -30,10 +31,16 @@
 // otherwise take cross-lane shuffles:
 //   recompute:      Σ_l dy_{t-1}[l] H_{t-1}[i, l] = dq_{t-1}[i]
 //   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
+// Software pipelining: the recompute of one chunk and the reverse walk of
+// the chunk after it (in time) are independent chains, so the epilogue
+// interleaves them step for step, each with its own TMEM accumulators, MMA
+// issuer warp and scratch buffer; each chain's MMA round trip overlaps the
+// other chain's epilogue work.
 // dv, df are thread-local plus shuffles; their per-warp partials are summed
-// in a fixed order by a storer warp, and the dW partials per (b, h) are
-// summed over the batch in a fixed order by a separate kernel, so results
-// are deterministic.
+// in a fixed order by a storer warp (with two slices, added into a zeroed
+// output, which is order-independent for two addends), and the dW partials
+// per CTA are summed over the batch and slices in a fixed order by a
+// separate kernel, so results are deterministic.
 //
 // Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16.
 #include <cuda_bf16.h>
@@ -44,9 +51,13 @@
 
 namespace m2rnn {
 
-template <int K_>
+// K state rows are handled as NSL independent slices of KS rows, one CTA
+// per (b, h, slice): the rows of H evolve independently given W, v_t and f_t,
+// so a slice needs only its own rows of k, q, the checkpoints and dH_T.
+template <int KS_, int NSL_>
 struct BwdTcCfg {
-    static constexpr int K = K_, V = 64;
+    static constexpr int K = KS_;             // rows of this CTA's slice
+    static constexpr int NSL = NSL_, KF = K * NSL, V = 64;
     static constexpr int P = 2;
     static constexpr int MPAD = 64;           // M of the dW MMA and of the state-operand layout
     static constexpr int MX = 128;            // M of the recompute and G-propagation MMAs
@@ -54,7 +65,7 @@ struct BwdTcCfg {
     static constexpr int R = K / P;           // rows per tile
     static constexpr int NT = 2 * R;          // MMA N per tile (hi rows, then lo rows)
     // two warps per TMEM lane quarter and tile (each owning half of the tile's
-    // rows) when the tile is large enough: the reverse step is issue-bound, and
+    // rows) when the tile is large enough: the epilogue is issue-bound, and
     // more warps with fewer rows each raise the issue rate
     static constexpr int SUBS = (R / 4 >= 4) ? 2 : 1;
     static constexpr int WPT = 4 * SUBS;      // epilogue warps per tile
@@ -62,14 +73,17 @@ struct BwdTcCfg {
     static constexpr int CMAX = 16;           // max steps per checkpoint chunk
     static constexpr int NWE = P * WPT;       // epilogue warps
     static constexpr int NSLOT = P * SUBS;    // dv partials per (t, j)
-    static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
-    static constexpr int NTHREADS = (NWE + 3) * 32;
+    // service warps; the two readers of TMEM lane XLANE sit in lane quarter 0
+    static constexpr int W_XD = NWE, W_MREV = NWE + 1, W_MREC = NWE + 2, W_STORE = NWE + 3, W_XQ = NWE + 4,
+                         W_PROD = NWE + 5;
+    static constexpr int NTHREADS = (NWE + 6) * 32;
+    static constexpr int NSTAGE = 3;          // input chunks: recompute of i, reverse of i-1, prefetch of i+1
 
     static constexpr int AX_BYTES = MX * V * 2;            // one extended A operand
     static constexpr int B_BYTES = NT * V * 2;
     static constexpr int ST_K = 0;
-    static constexpr int ST_Q = CMAX * K * 2;
-    static constexpr int ST_V = 2 * CMAX * K * 2;
+    static constexpr int ST_Q = CMAX * KF * 2;   // k and q rows hold all KF values
+    static constexpr int ST_V = 2 * CMAX * KF * 2;
     static constexpr int ST_DY = ST_V + CMAX * V * 2;      // CMAX + 1 rows: row r is step c0 - 1 + r
     static constexpr int ST_F = ST_DY + (CMAX + 1) * V * 2;
     static constexpr int STAGE_BYTES = ((ST_F + CMAX * 4) + 127) / 128 * 128;
@@ -79,22 +93,32 @@ struct BwdTcCfg {
 
     static constexpr int OFF_AF = 0;                       // Ã_f per tile (K-major)
     static constexpr int OFF_AG = OFF_AF + P * AX_BYTES;   // Ã_g per tile (MN-major)
-    static constexpr int OFF_BS = OFF_AG + P * AX_BYTES;   // state operands (recompute; H_{t-1} for dW)
+    static constexpr int OFF_BR = OFF_AG + P * AX_BYTES;   // recompute state operands
+    static constexpr int OFF_BS = OFF_BR + P * B_BYTES;    // H_{t-1} operands of the dW MMA
     static constexpr int OFF_BD = OFF_BS + P * B_BYTES;    // dA operands
     static constexpr int OFF_RING = OFF_BD + P * B_BYTES;
-    static constexpr int OFF_PART = OFF_RING + 2 * STAGE_BYTES;
-    static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
-    static constexpr int NBAR = 4 + 2 * P + 2;
+    static constexpr int OFF_CK = OFF_RING + NSTAGE * STAGE_BYTES;   // the next checkpoint (fp32 [K][V])
+    static constexpr int OFF_PART = OFF_CK + K * V * 4;
+    // dv / df partials: double-buffered when shared memory allows, so the
+    // storer's pass over one chunk overlaps the next chunk's reverse walk
+    static constexpr int NPART = (OFF_PART + 2 * PART_BYTES + 256 <= 227 * 1024) ? 2 : 1;
+    static constexpr int OFF_BAR = OFF_PART + NPART * PART_BYTES;
+    // in_full[3], in_empty[3], bready/accfull of both chains per tile, pfull/pempty per
+    // partial buffer, ck_full/ck_empty
+    static constexpr int NBAR = 2 * NSTAGE + 4 * P + 2 * NPART + 2;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
-    static constexpr int ACC_COLS = P * NT;                // per-tile accumulators
-    static constexpr int DW_COL = ACC_COLS;                // dW accumulator (V columns)
-    static constexpr int TMEM_COLS = (ACC_COLS + V <= 128) ? 128 : (ACC_COLS + V <= 256) ? 256 : 512;
+    static constexpr int REV_COL = 0;                      // G-propagation accumulators, NT columns per tile
+    static constexpr int REC_COL = P * NT;                 // recompute accumulators
+    static constexpr int DW_COL = 2 * P * NT;              // dW accumulator (V columns)
+    static constexpr int TMEM_COLS = (DW_COL + V <= 128) ? 128 : (DW_COL + V <= 256) ? 256 : 512;
 
-    static_assert(K == 32 || K == 64 || K == 128, "K");
+    static_assert(K == 32 || K == 64, "slice rows");
     static_assert(R % 16 == 0, "dW MMA needs 16-row k-steps");
     static_assert(NT % 16 == 0 && NT <= 256, "N of an M = 128 MMA");
     static_assert(RT % 4 == 0 && NWE * 32 * RT == K * V, "row split");
     static_assert(NTHREADS <= 1024, "block size");
+    static_assert(W_XD % 4 == 0 && W_XQ % 4 == 0, "lane-quarter 0 readers");
+    static_assert(DW_COL + V <= 512, "TMEM columns");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
 
@@ -135,39 +159,54 @@ __device__ __forceinline__ void store_xrow(uint32_t tcol, float* dst, bool store
     }
 }
 
-template <int K>
-__global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(const Params p) {
-    using C = BwdTcCfg<K>;
-    constexpr int V = C::V;
+template <int KS, int NSL>
+__global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_kernel(const Params p) {
+    using C = BwdTcCfg<KS, NSL>;
+    constexpr int K = C::K, KF = C::KF, V = C::V;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
+    const int bh = blockIdx.x / NSL;
+    const int koff = (blockIdx.x % NSL) * K;   // first state row of this slice
     const int hd = bh % p.H;
     const int T = p.T, CS = p.C;
     const int nck = (T + CS - 1) / CS;
 
+    // Chunks are processed in reverse time order; chunk i of that order is
+    // chunk c = nck-1-i of the sequence.  In phase m = 0 .. nck the epilogue
+    // walks chunk m-1 in reverse while it recomputes chunk m, step for step,
+    // so that each chain's MMA round trip overlaps the other chain's epilogue.
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     auto in_full = [&](int s) { return bar(s); };
-    auto in_empty = [&](int s) { return bar(2 + s); };
-    auto bready = [&](int t) { return bar(4 + t); };
-    auto accfull = [&](int t) { return bar(4 + C::P + t); };
-    const uint32_t pfull = bar(4 + 2 * C::P), pempty = bar(5 + 2 * C::P);
+    auto in_empty = [&](int s) { return bar(C::NSTAGE + s); };
+    auto bready_rev = [&](int t) { return bar(2 * C::NSTAGE + t); };
+    auto accfull_rev = [&](int t) { return bar(2 * C::NSTAGE + C::P + t); };
+    auto bready_rec = [&](int t) { return bar(2 * C::NSTAGE + 2 * C::P + t); };
+    auto accfull_rec = [&](int t) { return bar(2 * C::NSTAGE + 3 * C::P + t); };
+    auto pfull = [&](int b) { return bar(2 * C::NSTAGE + 4 * C::P + b); };
+    auto pempty = [&](int b) { return bar(2 * C::NSTAGE + 4 * C::P + C::NPART + b); };
+    const uint32_t ck_full = bar(2 * C::NSTAGE + 4 * C::P + 2 * C::NPART);
+    const uint32_t ck_empty = bar(2 * C::NSTAGE + 4 * C::P + 2 * C::NPART + 1);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* part = reinterpret_cast<float*>(smem + C::OFF_PART);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(in_full(s), 1);
             mbar_init(in_empty(s), C::NWE);
         }
         for (int t = 0; t < C::P; ++t) {
-            mbar_init(bready(t), C::WPT);
-            mbar_init(accfull(t), 1);
+            mbar_init(bready_rev(t), C::WPT + 1);   // epilogue warps + the dk reader
+            mbar_init(accfull_rev(t), 1);
+            mbar_init(bready_rec(t), C::WPT + 1);   // epilogue warps + the dq reader
+            mbar_init(accfull_rec(t), 1);
         }
-        mbar_init(pfull, C::NWE);
-        mbar_init(pempty, 1);
+        for (int b = 0; b < C::NPART; ++b) {
+            mbar_init(pfull(b), C::NWE);
+            mbar_init(pempty(b), 1);
+        }
+        mbar_init(ck_full, 1);
+        mbar_init(ck_empty, C::NWE);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -208,20 +247,25 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         const int nloc = nsub + half * C::RT;      // first tile row of this thread
         const int row0 = tile * C::R + nloc;
         const int slot = tile * C::SUBS + sub;
-        const bool xwriter = sub == 0 && half == 0;      // writes element j of the extra A rows
-        const bool xreader = sub == 0 && qd == 0;        // warp that reads TMEM lane XLANE
-        const size_t sbase = (size_t)bh * K * V;
+        const bool xwriter = sub == 0 && half == 0;            // writes element j of the extra A rows
+        const size_t sbase = ((size_t)bh * KF + koff) * V;   // this slice's rows of dH_T / dH0
+        uint8_t* Br = smem + C::OFF_BR + tile * C::B_BYTES;
         uint8_t* Bs = smem + C::OFF_BS + tile * C::B_BYTES;
         uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
         uint16_t* xf = reinterpret_cast<uint16_t*>(smem + C::OFF_AF + tile * C::AX_BYTES + af_off(C::XLANE, j));
         uint16_t* xg = reinterpret_cast<uint16_t*>(smem + C::OFF_AG + tile * C::AX_BYTES + ag_off(C::XLANE, j));
-        const uint32_t tcol = tmem + (uint32_t)(tile * C::NT);
-        const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT + nsub);
-        // Scratch, thread-contiguous: step u, thread t holds its RT values at
-        // u·K·V + t·RT (16-byte vector accesses, each warp touching one
-        // contiguous block).  Only the thread that wrote a value reads it back.
-        float* Sst = p.scratch + (size_t)bh * (2 * CS + 1) * K * V;   // states H_{c0+u}, u = 0..len
-        float* Sz = Sst + (size_t)(CS + 1) * K * V;                   // Z_{c0+u}, u = 0..len-1
+        const uint32_t lanes = (uint32_t)(qd * 32) << 16;
+        const uint32_t tb_rev = tmem + (uint32_t)(C::REV_COL + tile * C::NT + nsub) + lanes;
+        const uint32_t tb_rec = tmem + (uint32_t)(C::REC_COL + tile * C::NT + nsub) + lanes;
+        // Scratch, two buffers of (2C+1) states per CTA (the chunk being
+        // recomputed and the chunk being walked back): buffer b holds H_{c0+u}
+        // for u = 0..len, then Z_{c0+u} for u = 0..len-1.  Thread-contiguous:
+        // step u, thread t holds its RT values at u·K·V + t·RT (16-byte vector
+        // accesses, each warp touching one contiguous block); only the thread
+        // that wrote a value reads it back.
+        float* const Sc = p.scratch + (size_t)blockIdx.x * 2 * (2 * CS + 1) * K * V;
+        auto Sst = [&](int b) { return Sc + (size_t)b * (2 * CS + 1) * K * V; };
+        auto Sz = [&](int b) { return Sst(b) + (size_t)(CS + 1) * K * V; };
         const size_t tslot = (size_t)threadIdx.x * C::RT;
         auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
             float4* d = reinterpret_cast<float4*>(base + (size_t)u * K * V + tslot);
@@ -236,54 +280,134 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
             }
         };
-        // Row t of dq or dk for this tile's rows, from TMEM lane XLANE (reader
-        // warp only; nothing is stored for t < 0).
-        auto emit_xrow = [&](float* out, int t) {
-            store_xrow<C>(tcol, out + ((size_t)bh * T + max(t, 0)) * K + tile * C::R, lane == C::XLANE && t >= 0);
-        };
+        auto stage = [&](int i) { return smem + C::OFF_RING + (i % C::NSTAGE) * C::STAGE_BYTES; };
 
-        float G[C::RT];
+        float G[C::RT], h[C::RT], zc[C::RT], hpc[C::RT];
 #pragma unroll
         for (int r = 0; r < C::RT; ++r) G[r] = p.dHT != nullptr ? p.dHT[sbase + (size_t)(row0 + r) * V + j] : 0.f;
         float fprev = 0.f;
-        uint32_t nacc = 0;
+        uint32_t nrev = 0, nrec = 0;   // accumulator-full events consumed per chain
         bool ok = true;
-        for (int ci = 0; ci < nck && ok; ++ci) {
-            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0), s = ci & 1;
-            // the chunk holding step T-1 runs one more recompute MMA, for dq_{T-1} = H_{T-1} dy_{T-1}
-            const int nmma = len + (ci == 0 ? 1 : 0);
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (ci >> 1) & 1, abort_flag, p));
-            if (!ok) break;
-            const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
-            // dy of step c0 + u, for u = -1 .. len-1 (row -1 only when c0 > 0)
-            auto dy_row = [&](int u) { return reinterpret_cast<const uint16_t*>(st + C::ST_DY + (u + 1) * V * 2); };
-            // ------------------------------------------------ recompute the chunk
-            {
-                float h[C::RT];
-                const float* ck = p.ckpt + ((size_t)bh * nck + c) * K * V;
+        for (int m = 0; m <= nck && ok; ++m) {
+            // recompute: chunk m of the processing order (the chunk holding step
+            // T-1 runs one more MMA, for dq_{T-1} = H_{T-1} dy_{T-1})
+            const bool has_rec = m < nck;
+            const int c0r = (nck - 1 - m) * CS;
+            const int lenr = has_rec ? min(CS, T - c0r) : 0;
+            const int nmr = has_rec ? lenr + (m == 0 ? 1 : 0) : 0;
+            const uint8_t* str = stage(m);
+            float* const Sst_r = Sst(m & 1);
+            float* const Sz_r = Sz(m & 1);
+            // reverse: chunk m-1
+            const bool has_rev = m >= 1;
+            const int c0v = (nck - m) * CS;
+            const int lenv = has_rev ? min(CS, T - c0v) : 0;
+            const uint8_t* stv = stage(m + C::NSTAGE - 1);
+            const float* const Sst_v = Sst((m + 1) & 1);
+            const float* const Sz_v = Sz((m + 1) & 1);
+            const int pb = (m + C::NPART - 1) % C::NPART;   // partial-sum buffer of chunk m-1
+            float* const part = reinterpret_cast<float*>(smem + C::OFF_PART + pb * C::PART_BYTES);
+            auto dyr = [&](int u) {   // dy of step c0r + u of the recompute chunk, u >= -1
+                return reinterpret_cast<const uint16_t*>(str + C::ST_DY + (u + 1) * V * 2);
+            };
+
+            if (has_rec) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(m % C::NSTAGE), (m / C::NSTAGE) & 1, abort_flag, p));
+                if (!ok) break;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(ck_full, m & 1, abort_flag, p));
+                if (!ok) break;
+                const float* ck = reinterpret_cast<const float*>(smem + C::OFF_CK);
 #pragma unroll
-                for (int r = 0; r < C::RT; ++r) h[r] = ck[(size_t)(row0 + r) * V + j];
-                st_vec(Sst, 0, h);
-                write_state_operand<C>(Bs, h, j, nloc);
-                if (xwriter) *xf = c0 > 0 ? dy_row(-1)[j] : (uint16_t)0;
+                for (int r = 0; r < C::RT; ++r) h[r] = ck[(row0 + r) * V + j];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(ck_empty);
+                st_vec(Sst_r, 0, h);
+                write_state_operand<C>(Br, h, j, nloc);
+                if (xwriter) *xf = c0r > 0 ? dyr(-1)[j] : (uint16_t)0;
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bready(tile));
-                for (int u = 0; u < nmma; ++u) {
-                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
+                if (lane == 0) mbar_arrive(bready_rec(tile));
+            }
+            if (has_rev) {
+                const int i = m - 1;
+                if (i >= C::NPART) {   // the storer is done with this buffer's previous chunk
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(pempty(pb), ((i / C::NPART) - 1) & 1, abort_flag, p));
                     if (!ok) break;
-                    ++nacc;
+                }
+                ld_vec(Sz_v, lenv - 1, zc);
+                ld_vec(Sst_v, lenv - 1, hpc);
+            }
+            const int nsteps = max(nmr, lenv);
+            for (int s = 0; s < nsteps; ++s) {
+                if (s < lenv) {
+                    // ---------------------------------------- reverse step t = c0v + u
+                    const int u = lenv - 1 - s;
+                    if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step; emit dk_{t+1}
+                        ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
+                        if (!ok) break;
+                        ++nrev;
+                        tc_fence_after();
+                        uint32_t dhi[C::RT], dlo[C::RT];
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
+                        tc_wait_ld();
+                        reg_fence(dhi);
+                        reg_fence(dlo);
+#pragma unroll
+                        for (int r = 0; r < C::RT; ++r)
+                            G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                        tc_fence_before();
+                    }
+                    const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(stv + C::ST_DY + (u + 1) * V * 2 + j * 2));
+                    const uint16_t vbits = *reinterpret_cast<const uint16_t*>(stv + C::ST_V + u * V * 2 + j * 2);
+                    const float ft = *reinterpret_cast<const float*>(stv + C::ST_F + u * 4);
+                    float qq[C::RT], kk[C::RT];
+                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_Q + u * KF * 2) + koff + row0, qq);
+                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_K + u * KF * 2) + koff + row0, kk);
+                    float dA[C::RT];
+                    float dfp = 0.f, dvp = 0.f;
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r) {
+                        const float z = zc[r];
+                        G[r] = fmaf(qq[r], dyj, G[r]);
+                        dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
+                        dfp = fmaf(G[r], hpc[r] - z, dfp);
+                        dvp = fmaf(dA[r], kk[r], dvp);
+                    }
+                    write_state_operand<C, true>(Bd, dA, j, nloc);
+                    write_state_operand<C, true>(Bs, hpc, j, nloc);
+                    if (xwriter) *xg = vbits;
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bready_rev(tile));
+                    if (u > 0) {
+                        ld_vec(Sz_v, u - 1, zc);
+                        ld_vec(Sst_v, u - 1, hpc);
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
+                    if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
+                    dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
+                    if (half == 0) part[(C::DVP / 4) + (u * C::NSLOT + slot) * V + j] = dvp;
+                    fprev = ft;
+                }
+                if (s < nmr) {
+                    // ---------------------------------------- recompute step c0r + u
+                    const int u = s;
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rec(tile), nrec & 1, abort_flag, p));
+                    if (!ok) break;
+                    ++nrec;
                     tc_fence_after();
-                    if (xreader) emit_xrow(p.dq, c0 + u - 1);
-                    if (u < len) {
+                    if (u < lenr) {
                         const float vj =
-                            bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2));
-                        const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
+                            bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(str + C::ST_V + u * V * 2 + j * 2));
+                        const float g = 1.f - *reinterpret_cast<const float*>(str + C::ST_F + u * 4);
                         uint32_t ahi[C::RT], alo[C::RT];
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tbase, ahi);
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, alo);
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec, ahi);
+                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec + C::R, alo);
                         float kk[C::RT];
-                        lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
+                        lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(str + C::ST_K + u * KF * 2) + koff + row0, kk);
                         tc_wait_ld();
                         reg_fence(ahi);
                         reg_fence(alo);
@@ -295,130 +419,102 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                             zz[r] = tanh_exp(a);
                             h[r] = fmaf(g, zz[r] - h[r], h[r]);
                         }
-                        st_vec(Sz, u, zz);
-                        st_vec(Sst, u + 1, h);
+                        st_vec(Sz_r, u, zz);
+                        if (u + 1 < lenr) st_vec(Sst_r, u + 1, h);   // H_{c0+len} is not read back
                     }
                     tc_fence_before();
-                    if (u + 1 < nmma) {
-                        write_state_operand<C>(Bs, h, j, nloc);
-                        if (xwriter) *xf = dy_row(u)[j];
+                    if (u + 1 < nmr) {
+                        write_state_operand<C>(Br, h, j, nloc);
+                        if (xwriter) *xf = dyr(u)[j];
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(bready(tile));
+                        if (lane == 0) mbar_arrive(bready_rec(tile));
                     }
                 }
-                if (!ok) break;
             }
-            // ------------------------------------------------ reverse over the chunk
-            if (ci >= 1) {
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(pempty, (ci - 1) & 1, abort_flag, p));
+            if (!ok) break;
+            if (has_rev) {
+                // G_{c0-1} = f_{c0} G_{c0} + dA_{c0} Wᵀ
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
                 if (!ok) break;
-            }
-            // scratch values of the step being processed: H_{t-1} and Z_t.  The
-            // next step's are loaded right after each step's arrive, so their L2
-            // latency overlaps the MMA round trip.
-            float zc[C::RT], hpc[C::RT];
-            ld_vec(Sz, len - 1, zc);
-            ld_vec(Sst, len - 1, hpc);
-            for (int u = len - 1; u >= 0; --u) {
-                if (u < len - 1) {   // fold in dA_{t+1} Wᵀ from the previous reverse step; emit dk_{t+1}
-                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
-                    if (!ok) break;
-                    ++nacc;
-                    tc_fence_after();
+                ++nrev;
+                tc_fence_after();
+                {
                     uint32_t dhi[C::RT], dlo[C::RT];
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase, dhi);
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, dlo);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
                     tc_wait_ld();
                     reg_fence(dhi);
                     reg_fence(dlo);
 #pragma unroll
                     for (int r = 0; r < C::RT; ++r)
                         G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
-                    if (xreader) emit_xrow(p.dk, c0 + u + 1);
-                    tc_fence_before();
                 }
-                const float dyj = bf16lo_to_f32(dy_row(u)[j]);
-                const uint16_t vbits = *reinterpret_cast<const uint16_t*>(st + C::ST_V + u * V * 2 + j * 2);
-                const float ft = *reinterpret_cast<const float*>(st + C::ST_F + u * 4);
-                float qq[C::RT], kk[C::RT];
-                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_Q + u * K * 2) + row0, qq);
-                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(st + C::ST_K + u * K * 2) + row0, kk);
-                float dA[C::RT];
-                float dfp = 0.f, dvp = 0.f;
-#pragma unroll
-                for (int r = 0; r < C::RT; ++r) {
-                    const float z = zc[r];
-                    G[r] = fmaf(qq[r], dyj, G[r]);
-                    dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
-                    dfp = fmaf(G[r], hpc[r] - z, dfp);
-                    dvp = fmaf(dA[r], kk[r], dvp);
-                }
-                write_state_operand<C, true>(Bd, dA, j, nloc);
-                write_state_operand<C, true>(Bs, hpc, j, nloc);
-                if (xwriter) *xg = vbits;
-                fence_proxy_async_smem();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bready(tile));
-                if (u > 0) {
-                    ld_vec(Sz, u - 1, zc);
-                    ld_vec(Sst, u - 1, hpc);
+                if (lane == 0) {
+                    mbar_arrive(in_empty((m - 1) % C::NSTAGE));
+                    mbar_arrive(pfull(pb));
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
-                if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
-                dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
-                if (half == 0) part[(C::DVP / 4) + (u * C::NSLOT + slot) * V + j] = dvp;
-                fprev = ft;
-            }
-            if (!ok) break;
-            // G_{c0-1} = f_{c0} G_{c0} + dA_{c0} Wᵀ; emit dk_{c0}
-            ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull(tile), nacc & 1, abort_flag, p));
-            if (!ok) break;
-            ++nacc;
-            tc_fence_after();
-            {
-                uint32_t dhi[C::RT], dlo[C::RT];
-                tmem_ld_16x32bx2<C::RT, C::RT>(tbase, dhi);
-                tmem_ld_16x32bx2<C::RT, C::RT>(tbase + C::R, dlo);
-                tc_wait_ld();
-                reg_fence(dhi);
-                reg_fence(dlo);
-#pragma unroll
-                for (int r = 0; r < C::RT; ++r)
-                    G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
-            }
-            if (xreader) emit_xrow(p.dk, c0);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(in_empty(s));
-                mbar_arrive(pfull);
             }
         }
         if (ok) {
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) p.dH0[sbase + (size_t)(row0 + r) * V + j] = G[r];
         }
+    } else if (warp == C::W_XD || warp == C::W_XQ) {
+        // ------------------------------------------------------------ dk / dq readers
+        // Each result of the G-propagation (W_XD) or recompute (W_XQ) MMAs of a
+        // tile is read here from TMEM lane XLANE before the tile's next MMA of
+        // that chain may be issued (this warp is one of the arrivals it waits
+        // for), off the epilogue warps' path.  G-propagation MMAs come per
+        // reverse step, t = c0+len-1 .. c0; recompute MMA u of a chunk yields
+        // dq_{c0+u-1}, and the chunk holding step T-1 runs one more of them.
+        const bool xd = warp == C::W_XD;
+        float* const out = xd ? p.dk : p.dq;
+        if (lane == 0)
+            for (int tile = 0; tile < C::P; ++tile) mbar_arrive(xd ? bready_rev(tile) : bready_rec(tile));
+        uint32_t ne = 0;
+        bool ok = true;
+        for (int i = 0; i < nck && ok; ++i) {
+            const int c0 = (nck - 1 - i) * CS, len = min(CS, T - c0);
+            const int nev = xd ? len : len + (i == 0 ? 1 : 0);
+            for (int e = 0; e < nev && ok; ++e, ++ne) {
+                const int t = xd ? c0 + len - 1 - e : c0 + e - 1;
+                const bool last = i == nck - 1 && e == nev - 1;
+                for (int tile = 0; tile < C::P; ++tile) {
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(xd ? accfull_rev(tile) : accfull_rec(tile), ne & 1,
+                                                                    abort_flag, p));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t tcol = tmem + (uint32_t)((xd ? C::REV_COL : C::REC_COL) + tile * C::NT);
+                    store_xrow<C>(tcol, out + ((size_t)bh * T + max(t, 0)) * KF + koff + tile * C::R,
+                                  lane == C::XLANE && t >= 0);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (!last && lane == 0) mbar_arrive(xd ? bready_rev(tile) : bready_rec(tile));
+                }
+            }
+        }
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer (chunks in reverse order)
-        int last = -1;
-        for (int ci = 0; ci < nck; ++ci) {
-            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0), s = ci & 1;
-            if (ci >= 2) {
-                const bool ok =
-                    __all_sync(0xffffffffu, mbar_wait_bounded(in_empty(s), ((ci >> 1) - 1) & 1, abort_flag, p));
+        int last = -1, last_ck = -1;   // last chunk whose inputs / checkpoint were requested
+        for (int i = 0; i < nck; ++i) {
+            const int c0 = (nck - 1 - i) * CS, len = min(CS, T - c0), s = i % C::NSTAGE;
+            if (i >= C::NSTAGE) {
+                const bool ok = __all_sync(
+                    0xffffffffu, mbar_wait_bounded(in_empty(s), ((i / C::NSTAGE) - 1) & 1, abort_flag, p));
                 if (!ok) break;
             }
             uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
             if (lane < len) reinterpret_cast<float*>(st + C::ST_F)[lane] = p.f[(size_t)bh * T + c0 + lane];
             __syncwarp();
             if (lane == 0) {
-                const uint32_t kb = (uint32_t)(len * K * 2), vb = (uint32_t)(len * V * 2);
+                const uint32_t kb = (uint32_t)(len * KF * 2), vb = (uint32_t)(len * V * 2);
                 // dy rows c0-1 .. c0+len-1; the row of step c0-1 exists only when c0 > 0
                 const uint32_t dyb = (uint32_t)((len + (c0 > 0 ? 1 : 0)) * V * 2);
                 mbar_arrive_expect_tx(in_full(s), 2 * kb + vb + dyb);
-                const size_t rk = ((size_t)bh * T + c0) * K, rv = ((size_t)bh * T + c0) * V;
+                const size_t rk = ((size_t)bh * T + c0) * KF, rv = ((size_t)bh * T + c0) * V;
                 const uint16_t* dyg = static_cast<const uint16_t*>(p.dy) + rv;
                 bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + rk, kb, in_full(s));
                 bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + rk, kb, in_full(s));
@@ -428,15 +524,30 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 else
                     bulk_g2s(smem_u32(st + C::ST_DY + V * 2), dyg, dyb, in_full(s));
             }
-            last = ci;
+            last = i;
+            // checkpoint H_{c0} of this slice, once every warp has read the previous one
+            if (i >= 1) {
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(ck_empty, (i - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(ck_full, (uint32_t)(K * V * 4));
+                const float* ck = p.ckpt + ((size_t)bh * nck + (nck - 1 - i)) * KF * V + (size_t)koff * V;
+                bulk_g2s(smem_u32(smem + C::OFF_CK), ck, (uint32_t)(K * V * 4), ck_full);
+            }
+            last_ck = i;
         }
-        if (lane == 0)
-            for (int ci = max(0, last - 1); ci <= last; ++ci) mbar_wait_drain(in_full(ci & 1), (ci >> 1) & 1, p);
-        __syncwarp();
-    } else if (warp == C::W_MMA) {
-        // ------------------------------------------------------------ MMA issuer
+        // on an abort, copies may still be in flight: wait for them (bounded)
+        // before the CTA's shared memory is released
         if (lane == 0) {
-            constexpr uint32_t idesc_f = idesc_bf16_f32(C::MX, C::NT, 0, 1);
+            for (int i = max(0, last - (C::NSTAGE - 1)); i <= last; ++i)
+                mbar_wait_drain(in_full(i % C::NSTAGE), (i / C::NSTAGE) & 1, p);
+            if (last_ck >= 0) mbar_wait_drain(ck_full, last_ck & 1, p);
+        }
+        __syncwarp();
+    } else if (warp == C::W_MREV) {
+        // ------------------------------------------------------------ MMA issuer: reverse chain
+        if (lane == 0) {
             constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::NT, 1, 1);
             constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
             uint32_t nbr[C::P];
@@ -447,75 +558,111 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
                 issued[i] = -1;
             }
             bool first_dw = true, ok = true;
-            for (int ci = 0; ci < nck && ok; ++ci) {
-                const int c = nck - 1 - ci, len = min(CS, T - c * CS);
-                const int nmma = len + (ci == 0 ? 1 : 0);
-                for (int u = 0; u < nmma + len && ok; ++u) {
-                    const bool rev = u >= nmma;
+            for (int i = 0; i < nck && ok; ++i) {
+                const int len = min(CS, T - (nck - 1 - i) * CS);
+                for (int u = 0; u < len && ok; ++u) {
 #pragma unroll
                     for (int tile = 0; tile < C::P; ++tile) {
-                        if (!mbar_wait_bounded(bready(tile), nbr[tile] & 1, abort_flag, p)) {
+                        if (!mbar_wait_bounded(bready_rev(tile), nbr[tile] & 1, abort_flag, p)) {
                             ok = false;
                             break;
                         }
                         ++nbr[tile];
                         tc_fence_after();
-                        const uint32_t af = smem_u32(smem + C::OFF_AF + tile * C::AX_BYTES);
                         const uint32_t ag = smem_u32(smem + C::OFF_AG + tile * C::AX_BYTES);
                         const uint32_t bs = smem_u32(smem + C::OFF_BS + tile * C::B_BYTES);
                         const uint32_t bd = smem_u32(smem + C::OFF_BD + tile * C::B_BYTES);
-                        const uint32_t dt = tmem + (uint32_t)(tile * C::NT);
-                        if (!rev) {
+                        const uint32_t dt = tmem + (uint32_t)(C::REV_COL + tile * C::NT);
 #pragma unroll
-                            for (int ks = 0; ks < V / 16; ++ks)
-                                tc_mma_f16_ss(dt, smem_desc(af + ks * 256, 128, V * 16),
-                                              smem_desc(bs + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_f,
-                                              ks > 0 ? 1u : 0u);
-                        } else {
+                        for (int ks = 0; ks < V / 16; ++ks)
+                            tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
+                                          smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
+                                          ks > 0 ? 1u : 0u);
 #pragma unroll
-                            for (int ks = 0; ks < V / 16; ++ks)
-                                tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
-                                              smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
-                                              ks > 0 ? 1u : 0u);
-#pragma unroll
-                            for (int ks = 0; ks < C::R / 16; ++ks) {
-                                tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::NT * 16),
-                                              smem_desc(bd + ks * 256, 128, C::NT * 16), idesc_w,
-                                              (first_dw && ks == 0) ? 0u : 1u);
-                            }
-                            first_dw = false;
-                        }
-                        tc_commit(accfull(tile));
+                        for (int ks = 0; ks < C::R / 16; ++ks)
+                            tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::NT * 16),
+                                          smem_desc(bd + ks * 256, 128, C::NT * 16), idesc_w,
+                                          (first_dw && ks == 0) ? 0u : 1u);
+                        first_dw = false;
+                        tc_commit(accfull_rev(tile));
                         issued[tile] = (int)(nbr[tile] - 1);
                     }
                 }
             }
 #pragma unroll
             for (int tile = 0; tile < C::P; ++tile)
-                if (issued[tile] >= 0) mbar_wait_drain(accfull(tile), (uint32_t)issued[tile] & 1, p);
+                if (issued[tile] >= 0) mbar_wait_drain(accfull_rev(tile), (uint32_t)issued[tile] & 1, p);
+        }
+        __syncwarp();
+    } else if (warp == C::W_MREC) {
+        // ------------------------------------------------------------ MMA issuer: recompute chain
+        if (lane == 0) {
+            constexpr uint32_t idesc_f = idesc_bf16_f32(C::MX, C::NT, 0, 1);
+            uint32_t nbr[C::P];
+            int issued[C::P];
+#pragma unroll
+            for (int i = 0; i < C::P; ++i) {
+                nbr[i] = 0;
+                issued[i] = -1;
+            }
+            bool ok = true;
+            for (int i = 0; i < nck && ok; ++i) {
+                const int nm = min(CS, T - (nck - 1 - i) * CS) + (i == 0 ? 1 : 0);
+                for (int u = 0; u < nm && ok; ++u) {
+#pragma unroll
+                    for (int tile = 0; tile < C::P; ++tile) {
+                        if (!mbar_wait_bounded(bready_rec(tile), nbr[tile] & 1, abort_flag, p)) {
+                            ok = false;
+                            break;
+                        }
+                        ++nbr[tile];
+                        tc_fence_after();
+                        const uint32_t af = smem_u32(smem + C::OFF_AF + tile * C::AX_BYTES);
+                        const uint32_t br = smem_u32(smem + C::OFF_BR + tile * C::B_BYTES);
+                        const uint32_t dt = tmem + (uint32_t)(C::REC_COL + tile * C::NT);
+#pragma unroll
+                        for (int ks = 0; ks < V / 16; ++ks)
+                            tc_mma_f16_ss(dt, smem_desc(af + ks * 256, 128, V * 16),
+                                          smem_desc(br + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_f,
+                                          ks > 0 ? 1u : 0u);
+                        tc_commit(accfull_rec(tile));
+                        issued[tile] = (int)(nbr[tile] - 1);
+                    }
+                }
+            }
+#pragma unroll
+            for (int tile = 0; tile < C::P; ++tile)
+                if (issued[tile] >= 0) mbar_wait_drain(accfull_rec(tile), (uint32_t)issued[tile] & 1, p);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ dv / df storer
-        for (int ci = 0; ci < nck; ++ci) {
-            const int c = nck - 1 - ci, c0 = c * CS, len = min(CS, T - c0);
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull, ci & 1, abort_flag, p));
+        for (int i = 0; i < nck; ++i) {
+            const int c0 = (nck - 1 - i) * CS, len = min(CS, T - c0), b = i % C::NPART;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(pfull(b), (i / C::NPART) & 1, abort_flag, p));
             if (!ok) break;
+            const float* part = reinterpret_cast<const float*>(smem + C::OFF_PART + b * C::PART_BYTES);
             for (int e = lane; e < len * V; e += 32) {
                 const int u = e / V, jj = e % V;
                 float sv = 0.f;
 #pragma unroll
                 for (int sl = 0; sl < C::NSLOT; ++sl) sv += part[C::DVP / 4 + (u * C::NSLOT + sl) * V + jj];
-                p.dv[((size_t)bh * T + c0 + u) * V + jj] = sv;
+                float* dst = p.dv + ((size_t)bh * T + c0 + u) * V + jj;
+                // with two slices, the two partial sums meet in a zeroed output:
+                // 0 + a + b == 0 + b + a exactly, so the order does not matter
+                if constexpr (NSL == 1) *dst = sv;
+                else atomicAdd(dst, sv);
             }
             if (lane < len) {
                 float sf = 0.f;
 #pragma unroll
                 for (int w = 0; w < C::NWE; ++w) sf += part[C::DFP / 4 + lane * C::NWE + w];
-                p.df[(size_t)bh * T + c0 + lane] = sf;
+                float* dst = p.df + (size_t)bh * T + c0 + lane;
+                if constexpr (NSL == 1) *dst = sf;
+                else atomicAdd(dst, sf);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(pempty);
+            if (lane == 0) mbar_arrive(pempty(b));
         }
     }
 
@@ -529,7 +676,7 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
         tc_wait_ld();
         reg_fence(w);
         const int l = warp * 16 + (lane & 15), j0 = (lane >> 4) * 32;
-        float* dst = p.dW_part + ((size_t)bh * V + l) * V + j0;
+        float* dst = p.dW_part + ((size_t)blockIdx.x * V + l) * V + j0;
 #pragma unroll
         for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(w[e]), __uint_as_float(w[e + 1]),
@@ -543,33 +690,49 @@ __global__ void __launch_bounds__(BwdTcCfg<K>::NTHREADS, 1) m2rnn_bwd_tc_kernel(
     }
 }
 
-template <int K>
-static cudaError_t launch_bwd_tc_k(const Params& p, cudaStream_t stream) {
-    using C = BwdTcCfg<K>;
-    auto kern = m2rnn_bwd_tc_kernel<K>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+template <int KS, int NSL>
+static cudaError_t launch_bwd_tc_k(const Params& p0, cudaStream_t stream) {
+    using C = BwdTcCfg<KS, NSL>;
+    static_assert(NSL <= 2, "slice partial sums are exact for two addends only");
+    Params p = p0;
+    p.dw_parts = NSL;   // one dW partial per slice
+    cudaError_t e;
+    if (NSL > 1) {   // dv and df are summed over the slices
+        e = cudaMemsetAsync(p.dv, 0, sizeof(float) * (size_t)p.B * p.H * p.T * p.V, stream);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(p.df, 0, sizeof(float) * (size_t)p.B * p.H * p.T, stream);
+        if (e != cudaSuccess) return e;
+    }
+    auto kern = m2rnn_bwd_tc_kernel<KS, NSL>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<p.B * p.H, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    kern<<<p.B * p.H * NSL, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_dw_reduce(p, stream);
 }
 
+int bwd_tc_slices(int K) { return K > 64 ? 2 : 1; }
+
 bool bwd_tc_supported(int K, int V, int C) {
-    return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64>::CMAX;
+    return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64, 1>::CMAX;
 }
 
+// Per (b, h): dW partials of each slice, and two recompute buffers of
+// (2C+1)·K·V values (a chunk's states and Z's, for the chunk being
+// recomputed and the chunk being walked back).
 size_t bwd_tc_workspace(int B, int H, int K, int V, int C) {
     if (!bwd_tc_supported(K, V, C)) return 0;
-    return sizeof(float) * ((size_t)B * H * V * V + (size_t)B * H * (2 * C + 1) * K * V);
+    const size_t nsl = (size_t)bwd_tc_slices(K);
+    return sizeof(float) * ((size_t)B * H * nsl * V * V + (size_t)B * H * 2 * (2 * C + 1) * K * V);
 }
 
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s) {
     if (!bwd_tc_supported(p.K, p.V, p.C)) return cudaErrorNotSupported;
     switch (p.K) {
-        case 32: return launch_bwd_tc_k<32>(p, s);
-        case 64: return launch_bwd_tc_k<64>(p, s);
-        case 128: return launch_bwd_tc_k<128>(p, s);
+        case 32: return launch_bwd_tc_k<32, 1>(p, s);
+        case 64: return launch_bwd_tc_k<64, 1>(p, s);
+        case 128: return launch_bwd_tc_k<64, 2>(p, s);
     }
     return cudaErrorNotSupported;
 }

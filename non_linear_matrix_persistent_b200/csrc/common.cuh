@@ -34,7 +34,8 @@ struct Params {
     float* df;
     float* dW;
     float* dH0;
-    float* dW_part;     // [B*H][V][V] partial dW (workspace)
+    float* dW_part;     // [B*H][dw_parts][V][V] partial dW (workspace)
+    int dw_parts;       // dW partials per (b, h)
     float* scratch;     // per-CTA recompute scratch (workspace)
     uint32_t* status;   // device status word (workspace)
     uint64_t wait_limit_ns;

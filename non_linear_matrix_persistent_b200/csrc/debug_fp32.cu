@@ -187,7 +187,8 @@ __global__ void m2rnn_dw_reduce_kernel(const Params p) {
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
         const size_t h = e / VV, r = e % VV;
         float s = 0.f;
-        for (int b = 0; b < p.B; ++b) s += p.dW_part[((size_t)b * p.H + h) * VV + r];
+        for (int b = 0; b < p.B; ++b)
+            for (int sl = 0; sl < p.dw_parts; ++sl) s += p.dW_part[(((size_t)b * p.H + h) * p.dw_parts + sl) * VV + r];
         p.dW[e] = s;
     }
 }

@@ -20,6 +20,8 @@ cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
 // Shapes the tensor-core backward supports (V = 64, K in {32, 64, 128},
 // checkpoint stride <= 16).
 bool bwd_tc_supported(int K, int V, int C);
+// Row slices (CTAs per (b, h)) of the tensor-core backward for K state rows.
+int bwd_tc_slices(int K);
 
 // Workspace bytes beyond the 256-byte status header.
 size_t bwd_fp32_workspace(int B, int H, int K, int V, int C);

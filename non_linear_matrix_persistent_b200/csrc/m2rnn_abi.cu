@@ -32,6 +32,7 @@ m2rnn::Params base_params(const m2rnn_dims* d, void* ws) {
     p.status = static_cast<uint32_t*>(ws);
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.load();
+    p.dw_parts = 1;
     return p;
 }
 
@@ -116,7 +117,8 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     p.dy = dy; p.dHT = dHT; p.dk = dk; p.dv = dv; p.dq = dq; p.df = df; p.dW = dW; p.dH0 = dH0;
     uint8_t* extra = static_cast<uint8_t*>(workspace) + kStatusBytes;
     p.dW_part = reinterpret_cast<float*>(extra);
-    p.scratch = p.dW_part + (size_t)d->B * d->H * d->V * d->V;
+    p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K);
+    p.scratch = p.dW_part + (size_t)d->B * d->H * p.dw_parts * d->V * d->V;
     cudaError_t e = d->mode == M2RNN_MODE_FP32_DEBUG ? m2rnn::launch_bwd_fp32(p, s) : m2rnn::launch_bwd_tc(p, s);
     if (e == cudaErrorNotSupported) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return e == cudaSuccess ? M2RNN_OK : M2RNN_ERR_CUDA;
