@@ -33,9 +33,9 @@
 //   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
 // Software pipelining: the recompute of one chunk and the reverse walk of
 // the chunk after it (in time) are independent chains, so the epilogue
-// interleaves them step for step, each with its own TMEM accumulators, MMA
-// issuer warp and scratch buffer; each chain's MMA round trip overlaps the
-// other chain's epilogue work.
+// interleaves them step for step, each with its own TMEM accumulators and
+// MMA issuer warp, sharing one scratch buffer; each chain's MMA round trip
+// overlaps the other chain's epilogue work.
 // dv, df are thread-local plus shuffles; their per-warp partials are summed
 // in a fixed order by a storer warp (with two slices, added into a zeroed
 // output, which is order-independent for two addends), and the dW partials
@@ -257,20 +257,28 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         const uint32_t lanes = (uint32_t)(qd * 32) << 16;
         const uint32_t tb_rev = tmem + (uint32_t)(C::REV_COL + tile * C::NT + nsub) + lanes;
         const uint32_t tb_rec = tmem + (uint32_t)(C::REC_COL + tile * C::NT + nsub) + lanes;
-        // Scratch, two buffers of (2C+1) states per CTA (the chunk being
-        // recomputed and the chunk being walked back): buffer b holds H_{c0+u}
-        // for u = 0..len, then Z_{c0+u} for u = 0..len-1.  Thread-contiguous:
-        // step u, thread t holds its RT values at u·K·V + t·RT (16-byte vector
+        // Scratch per CTA: C slots of states (H_{c0+u}, the state before step
+        // c0+u) and C slots of Z_{c0+u}.  One buffer serves both chains: the
+        // chunk recomputed in phase i stores step u in slot u for even i and in
+        // slot C-1-u for odd i, so in phase i+1 the recompute writes exactly
+        // the slots the reverse walk (which reads its chunk from step len-1
+        // down, one step ahead) has already read.  Thread-contiguous: slot x,
+        // thread t holds its RT values at x·K·V + t·RT (16-byte vector
         // accesses, each warp touching one contiguous block); only the thread
         // that wrote a value reads it back.
-        float* const Sc = p.scratch + (size_t)blockIdx.x * 2 * (2 * CS + 1) * K * V;
-        auto Sst = [&](int b) { return Sc + (size_t)b * (2 * CS + 1) * K * V; };
-        auto Sz = [&](int b) { return Sst(b) + (size_t)(CS + 1) * K * V; };
+        float* const Sst = p.scratch + (size_t)blockIdx.x * 2 * CS * K * V;
+        float* const Sz = Sst + (size_t)CS * K * V;
+        auto sslot = [&](int i, int u) { return (i & 1) ? CS - 1 - u : u; };
         const size_t tslot = (size_t)threadIdx.x * C::RT;
+        // The scratch (2·C·K·V·4 bytes per CTA, ~64 MB for 128 CTAs at C = 16,
+        // K = V = 64) is stored with L2 evict_last priority, so its round trip
+        // stays in L2 instead of being written back to HBM and read again.
+        const uint64_t pol_keep = l2_policy_evict_last();
         auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
-            float4* d = reinterpret_cast<float4*>(base + (size_t)u * K * V + tslot);
+            float* d = base + (size_t)u * K * V + tslot;
 #pragma unroll
-            for (int g = 0; g < C::RT / 4; ++g) d[g] = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            for (int g = 0; g < C::RT / 4; ++g)
+                st_global_v4_hint(d + 4 * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3], pol_keep);
         };
         auto ld_vec = [&](const float* base, int u, float (&v)[C::RT]) {
             const float4* s4 = reinterpret_cast<const float4*>(base + (size_t)u * K * V + tslot);
@@ -296,21 +304,28 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
             const int lenr = has_rec ? min(CS, T - c0r) : 0;
             const int nmr = has_rec ? lenr + (m == 0 ? 1 : 0) : 0;
             const uint8_t* str = stage(m);
-            float* const Sst_r = Sst(m & 1);
-            float* const Sz_r = Sz(m & 1);
             // reverse: chunk m-1
             const bool has_rev = m >= 1;
             const int c0v = (nck - m) * CS;
             const int lenv = has_rev ? min(CS, T - c0v) : 0;
             const uint8_t* stv = stage(m + C::NSTAGE - 1);
-            const float* const Sst_v = Sst((m + 1) & 1);
-            const float* const Sz_v = Sz((m + 1) & 1);
             const int pb = (m + C::NPART - 1) % C::NPART;   // partial-sum buffer of chunk m-1
             float* const part = reinterpret_cast<float*>(smem + C::OFF_PART + pb * C::PART_BYTES);
             auto dyr = [&](int u) {   // dy of step c0r + u of the recompute chunk, u >= -1
                 return reinterpret_cast<const uint16_t*>(str + C::ST_DY + (u + 1) * V * 2);
             };
 
+            if (has_rev) {
+                const int i = m - 1;
+                if (i >= C::NPART) {   // the storer is done with this buffer's previous chunk
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(pempty(pb), ((i / C::NPART) - 1) & 1, abort_flag, p));
+                    if (!ok) break;
+                }
+                // before the recompute below stores its first state (same slot)
+                ld_vec(Sz, sslot(m - 1, lenv - 1), zc);
+                ld_vec(Sst, sslot(m - 1, lenv - 1), hpc);
+            }
             if (has_rec) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(m % C::NSTAGE), (m / C::NSTAGE) & 1, abort_flag, p));
                 if (!ok) break;
@@ -321,29 +336,19 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 for (int r = 0; r < C::RT; ++r) h[r] = ck[(row0 + r) * V + j];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ck_empty);
-                st_vec(Sst_r, 0, h);
+                st_vec(Sst, sslot(m, 0), h);
                 write_state_operand<C>(Br, h, j, nloc);
                 if (xwriter) *xf = c0r > 0 ? dyr(-1)[j] : (uint16_t)0;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rec(tile));
             }
-            if (has_rev) {
-                const int i = m - 1;
-                if (i >= C::NPART) {   // the storer is done with this buffer's previous chunk
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait_bounded(pempty(pb), ((i / C::NPART) - 1) & 1, abort_flag, p));
-                    if (!ok) break;
-                }
-                ld_vec(Sz_v, lenv - 1, zc);
-                ld_vec(Sst_v, lenv - 1, hpc);
-            }
             const int nsteps = max(nmr, lenv);
             for (int s = 0; s < nsteps; ++s) {
                 if (s < lenv) {
                     // ---------------------------------------- reverse step t = c0v + u
                     const int u = lenv - 1 - s;
-                    if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step; emit dk_{t+1}
+                    if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
                         ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
                         if (!ok) break;
                         ++nrev;
@@ -382,8 +387,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bready_rev(tile));
                     if (u > 0) {
-                        ld_vec(Sz_v, u - 1, zc);
-                        ld_vec(Sst_v, u - 1, hpc);
+                        ld_vec(Sz, sslot(m - 1, u - 1), zc);
+                        ld_vec(Sst, sslot(m - 1, u - 1), hpc);
                     }
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
@@ -419,8 +424,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                             zz[r] = tanh_exp(a);
                             h[r] = fmaf(g, zz[r] - h[r], h[r]);
                         }
-                        st_vec(Sz_r, u, zz);
-                        if (u + 1 < lenr) st_vec(Sst_r, u + 1, h);   // H_{c0+len} is not read back
+                        st_vec(Sz, sslot(m, u), zz);
+                        if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
                     }
                     tc_fence_before();
                     if (u + 1 < nmr) {
@@ -718,13 +723,12 @@ bool bwd_tc_supported(int K, int V, int C) {
     return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64, 1>::CMAX;
 }
 
-// Per (b, h): dW partials of each slice, and two recompute buffers of
-// (2C+1)·K·V values (a chunk's states and Z's, for the chunk being
-// recomputed and the chunk being walked back).
+// Per (b, h): dW partials of each slice, and the recompute scratch of
+// 2·C·K·V values (C states and C Z's of a chunk).
 size_t bwd_tc_workspace(int B, int H, int K, int V, int C) {
     if (!bwd_tc_supported(K, V, C)) return 0;
     const size_t nsl = (size_t)bwd_tc_slices(K);
-    return sizeof(float) * ((size_t)B * H * nsl * V * V + (size_t)B * H * 2 * (2 * C + 1) * K * V);
+    return sizeof(float) * ((size_t)B * H * nsl * V * V + (size_t)B * H * 2 * C * K * V);
 }
 
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s) {

@@ -79,26 +79,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
         : "memory");
 }
 
-// Same, with an L2 cache policy (createpolicy) for the source lines.
-__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
-                                              uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(dst),
-        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
-        : "memory");
-}
-
 // ---------------------------------------------------------------- L2 policies
-// Cache policies for accesses with .L2::cache_hint: lines of data that is
-// re-read soon (evict_last) or read / written once (evict_first).
+// Cache policy for accesses with .L2::cache_hint: lines of data that is
+// re-read soon are evicted last.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
 __device__ __forceinline__ void st_global_v4_hint(float* dst, float a, float b, float c, float d, uint64_t policy) {
@@ -106,13 +92,6 @@ __device__ __forceinline__ void st_global_v4_hint(float* dst, float a, float b, 
                  "f"(d), "l"(policy)
                  : "memory");
 }
-// Drops the 128-byte L2 line at p (128-byte aligned) without writing it
-// back: its contents become undefined.  For scratch that is dead after its
-// last read, so that dirty lines are not written back to HBM.
-__device__ __forceinline__ void discard_l2_line(const void* p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
-
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
