@@ -343,99 +343,108 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rec(tile));
             }
-            const int nsteps = max(nmr, lenv);
-            for (int s = 0; s < nsteps; ++s) {
-                if (s < lenv) {
-                    // ---------------------------------------- reverse step t = c0v + u
-                    const int u = lenv - 1 - s;
-                    if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
-                        ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
-                        if (!ok) break;
-                        ++nrev;
-                        tc_fence_after();
-                        uint32_t dhi[C::RT], dlo[C::RT];
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
-                        tc_wait_ld();
-                        reg_fence(dhi);
-                        reg_fence(dlo);
+            // one reverse step (chain step s of the phase) of this tile
+            auto rev_step = [&](int s) -> bool {
+                // ---------------------------------------- reverse step t = c0v + u
+                const int u = lenv - 1 - s;
+                if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
+                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
+                    if (!ok) return false;
+                    ++nrev;
+                    tc_fence_after();
+                    uint32_t dhi[C::RT], dlo[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
+                    tc_wait_ld();
+                    reg_fence(dhi);
+                    reg_fence(dlo);
 #pragma unroll
-                        for (int r = 0; r < C::RT; ++r)
-                            G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
-                        tc_fence_before();
-                    }
-                    const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(stv + C::ST_DY + (u + 1) * V * 2 + j * 2));
-                    const uint16_t vbits = *reinterpret_cast<const uint16_t*>(stv + C::ST_V + u * V * 2 + j * 2);
-                    const float ft = *reinterpret_cast<const float*>(stv + C::ST_F + u * 4);
-                    float qq[C::RT], kk[C::RT];
-                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_Q + u * KF * 2) + koff + row0, qq);
-                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_K + u * KF * 2) + koff + row0, kk);
-                    float dA[C::RT];
-                    float dfp = 0.f, dvp = 0.f;
+                    for (int r = 0; r < C::RT; ++r)
+                        G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                    tc_fence_before();
+                }
+                const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(stv + C::ST_DY + (u + 1) * V * 2 + j * 2));
+                const uint16_t vbits = *reinterpret_cast<const uint16_t*>(stv + C::ST_V + u * V * 2 + j * 2);
+                const float ft = *reinterpret_cast<const float*>(stv + C::ST_F + u * 4);
+                float qq[C::RT], kk[C::RT];
+                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_Q + u * KF * 2) + koff + row0, qq);
+                lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(stv + C::ST_K + u * KF * 2) + koff + row0, kk);
+                float dA[C::RT];
+                float dfp = 0.f, dvp = 0.f;
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) {
+                    const float z = zc[r];
+                    G[r] = fmaf(qq[r], dyj, G[r]);
+                    dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
+                    dfp = fmaf(G[r], hpc[r] - z, dfp);
+                    dvp = fmaf(dA[r], kk[r], dvp);
+                }
+                write_state_operand<C, true>(Bd, dA, j, nloc);
+                write_state_operand_hi<C>(Bs, hpc, j, nloc);   // the dW MMA reads the hi half only
+                if (xwriter) *xg = vbits;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bready_rev(tile));
+                if (u > 0) {
+                    ld_vec(Sz, sslot(m - 1, u - 1), zc);
+                    ld_vec(Sst, sslot(m - 1, u - 1), hpc);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
+                if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
+                dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
+                if (half == 0) part[(C::DVP / 4) + (u * C::NSLOT + slot) * V + j] = dvp;
+                fprev = ft;
+                return true;
+            };
+            // one recompute step (after the reverse step of the same s, which may
+            // still have to read the scratch slot this one writes)
+            auto rec_step = [&](int s) -> bool {
+                // ---------------------------------------- recompute step c0r + u
+                const int u = s;
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rec(tile), nrec & 1, abort_flag, p));
+                if (!ok) return false;
+                ++nrec;
+                tc_fence_after();
+                if (u < lenr) {
+                    const float vj =
+                        bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(str + C::ST_V + u * V * 2 + j * 2));
+                    const float g = 1.f - *reinterpret_cast<const float*>(str + C::ST_F + u * 4);
+                    uint32_t ahi[C::RT], alo[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec, ahi);
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec + C::R, alo);
+                    float kk[C::RT];
+                    lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(str + C::ST_K + u * KF * 2) + koff + row0, kk);
+                    tc_wait_ld();
+                    reg_fence(ahi);
+                    reg_fence(alo);
+                    float zz[C::RT];
 #pragma unroll
                     for (int r = 0; r < C::RT; ++r) {
-                        const float z = zc[r];
-                        G[r] = fmaf(qq[r], dyj, G[r]);
-                        dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
-                        dfp = fmaf(G[r], hpc[r] - z, dfp);
-                        dvp = fmaf(dA[r], kk[r], dvp);
+                        float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
+                        a = fmaf(kk[r], vj, a);
+                        zz[r] = tanh_exp(a);
+                        h[r] = fmaf(g, zz[r] - h[r], h[r]);
                     }
-                    write_state_operand<C, true>(Bd, dA, j, nloc);
-                    write_state_operand<C, true>(Bs, hpc, j, nloc);
-                    if (xwriter) *xg = vbits;
+                    st_vec(Sz, sslot(m, u), zz);
+                    if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
+                }
+                tc_fence_before();
+                if (u + 1 < nmr) {
+                    write_state_operand<C>(Br, h, j, nloc);
+                    if (xwriter) *xf = dyr(u)[j];
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bready_rev(tile));
-                    if (u > 0) {
-                        ld_vec(Sz, sslot(m - 1, u - 1), zc);
-                        ld_vec(Sst, sslot(m - 1, u - 1), hpc);
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
-                    if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
-                    dvp += __shfl_xor_sync(0xffffffffu, dvp, 16);
-                    if (half == 0) part[(C::DVP / 4) + (u * C::NSLOT + slot) * V + j] = dvp;
-                    fprev = ft;
+                    if (lane == 0) mbar_arrive(bready_rec(tile));
                 }
-                if (s < nmr) {
-                    // ---------------------------------------- recompute step c0r + u
-                    const int u = s;
-                    ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rec(tile), nrec & 1, abort_flag, p));
-                    if (!ok) break;
-                    ++nrec;
-                    tc_fence_after();
-                    if (u < lenr) {
-                        const float vj =
-                            bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(str + C::ST_V + u * V * 2 + j * 2));
-                        const float g = 1.f - *reinterpret_cast<const float*>(str + C::ST_F + u * 4);
-                        uint32_t ahi[C::RT], alo[C::RT];
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec, ahi);
-                        tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec + C::R, alo);
-                        float kk[C::RT];
-                        lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(str + C::ST_K + u * KF * 2) + koff + row0, kk);
-                        tc_wait_ld();
-                        reg_fence(ahi);
-                        reg_fence(alo);
-                        float zz[C::RT];
-#pragma unroll
-                        for (int r = 0; r < C::RT; ++r) {
-                            float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
-                            a = fmaf(kk[r], vj, a);
-                            zz[r] = tanh_exp(a);
-                            h[r] = fmaf(g, zz[r] - h[r], h[r]);
-                        }
-                        st_vec(Sz, sslot(m, u), zz);
-                        if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
-                    }
-                    tc_fence_before();
-                    if (u + 1 < nmr) {
-                        write_state_operand<C>(Br, h, j, nloc);
-                        if (xwriter) *xf = dyr(u)[j];
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bready_rec(tile));
-                    }
-                }
+                return true;
+            };
+            // (Running the chains in opposite orders on the two tiles, to spread
+            // the tanh bursts, was measured 16% slower.)
+            const int nsteps = max(nmr, lenv);
+            for (int s = 0; s < nsteps && ok; ++s) {
+                if (s < lenv) ok = rev_step(s);
+                if (ok && s < nmr) ok = rec_step(s);
             }
             if (!ok) break;
             if (has_rev) {

@@ -83,4 +83,26 @@ __device__ __forceinline__ void write_state_operand(uint8_t* Bt, const float (&h
     }
 }
 
+// Writes only the hi parts (bf16, round to nearest) of this thread's RT
+// values of column j, at n = nloc + r: for operands whose lo half no MMA reads.
+template <class C>
+__device__ __forceinline__ void write_state_operand_hi(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
+    uint8_t* colbase = Bt + (j >> 3) * (C::NT * 16) + (j & 7) * 16;
+    auto pack = [](float a, float b) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&v);
+    };
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g) {
+            const uint4 hi = make_uint4(pack(h[8 * g], h[8 * g + 1]), pack(h[8 * g + 2], h[8 * g + 3]),
+                                        pack(h[8 * g + 4], h[8 * g + 5]), pack(h[8 * g + 6], h[8 * g + 7]));
+            *reinterpret_cast<uint4*>(colbase + ((nloc + 8 * g) >> 3) * 128) = hi;
+        }
+    } else {
+        const uint2 hi = make_uint2(pack(h[0], h[1]), pack(h[2], h[3]));
+        *reinterpret_cast<uint2*>(colbase + (nloc >> 3) * 128 + (nloc & 7) * 2) = hi;
+    }
+}
+
 }  // namespace m2rnn
