@@ -120,7 +120,9 @@ class ClockSampler:
 
 
 def per_step_counts(w):
-    """Algorithmic work per (b, h, t) of each kernel (stated in the design doc §6)."""
+    """Algorithmic work per (b, h, t) of each kernel: tanh count, tensor FLOP
+    (one GEMM forward, three backward) and compulsory HBM bytes (bf16 inputs,
+    fp32 outputs and gradients, the fp32 checkpoint amortised over C steps)."""
     K, V, C = w.K, w.V, CKPT_STRIDE
     fwd = {"tanh": K * V, "flop": 2.0 * K * V * V,
            "bytes": (2 * K + V) * 2 + 4 + 4 * V + (4.0 * K * V / C if w.backward else 0.0)}

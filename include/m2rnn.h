@@ -78,11 +78,19 @@ typedef struct CUstream_st* m2rnn_stream_t;
 
 /* Bytes of device workspace a call needs (forward when backward == 0).
  * Returns 0 for invalid dims.  The first 256 bytes hold the device status
- * word: zero them once after allocating the workspace. */
+ * word: zero them once after allocating the workspace.  The rest is scratch
+ * the kernels write before they read it: for the backward, per-(b, h) dW
+ * partials and the chunk recompute buffer; for a tensor-core forward with
+ * few (b, h) pairs (B·H·2 <= 148), which splits each pair's K rows over
+ * several CTAs, the slices' partial readouts (slices · B·H·T·V fp32). */
 size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward);
 
 /* Forward scan.  H0 may be NULL (zero initial state).  HT (final state) and
- * ckpt (checkpoints for m2rnn_backward) may be NULL.  y is required. */
+ * ckpt (checkpoints for m2rnn_backward) may be NULL.  y is required.
+ * H0 and HT may be the same buffer: every element of H0 is read before the
+ * same element of HT is written, so the state can be advanced in place --
+ * with T = 1 this is one decode step, and T such calls give the scan's y and
+ * H_T bit for bit. */
 m2rnn_status m2rnn_forward(const m2rnn_dims* d,
                            const void* k, const void* v, const void* q,
                            const float* f, const void* W, const float* H0,
@@ -90,7 +98,8 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d,
                            void* workspace, size_t ws_bytes, m2rnn_stream_t stream);
 
 /* Backward through time for the loss L with dL/dy = dy and dL/dH_T = dHT
- * (NULL = 0).  ckpt must come from m2rnn_forward with the same inputs and
+ * (NULL = 0; dHT and dH0 may be the same buffer).  ckpt must come from
+ * m2rnn_forward with the same inputs and
  * the same dims (including ckpt_stride); the states inside each chunk of C
  * steps are recomputed from it.  Writes dk, dv, dq, df, dW, dH0 (all
  * required, all fp32).  M2RNN_MODE_BF16_TC supports V = 64, K in

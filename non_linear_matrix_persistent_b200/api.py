@@ -105,6 +105,24 @@ def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = 
     return y, HT, ckpt
 
 
+def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None):
+    """One decode step, in place: advances the fp32 state H [B, H, K, V] by one
+    step of the recurrence with k, q [B, H, K], v [B, H, V] and f [B, H], and
+    returns y [B, H, V].  It is the forward with T = 1 and the state buffer
+    passed as both H0 and H_T (the ABI allows that alias), so T calls give the
+    scan's outputs bit for bit."""
+    B, Hh, K = k.shape
+    V = v.shape[-1]
+    if H is None:
+        raise ValueError("step needs the state buffer H (it is updated in place)")
+    _check("H", H, (B, Hh, K, V), torch.float32, k.device)
+    if y is None:
+        y = torch.empty(B, Hh, V, dtype=torch.float32, device=k.device)
+    forward(k.unsqueeze(2), v.unsqueeze(2), q.unsqueeze(2), f.unsqueeze(2), W, H, ckpt_stride=1,
+            out={"y": y.view(B, Hh, 1, V), "HT": H})
+    return y
+
+
 def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: Optional[dict] = None):
     """BPTT from the forward's checkpoints.  Returns dict dk, dv, dq, df, dW, dH0 (fp32)."""
     dev = k.device

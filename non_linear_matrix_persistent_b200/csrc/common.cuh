@@ -36,6 +36,8 @@ struct Params {
     float* dH0;
     float* dW_part;     // [B*H][dw_parts][V][V] partial dW (workspace)
     int dw_parts;       // dW partials per (b, h)
+    int slices;         // forward: CTAs (row slices) per (b, h)
+    float* ypart;       // forward with slices > 1: [slices][B*H][T][V] partial readouts (workspace)
     float* scratch;     // per-CTA recompute scratch (workspace)
     uint32_t* status;   // device status word (workspace)
     uint64_t wait_limit_ns;

@@ -20,6 +20,10 @@ cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
 // Shapes the tensor-core backward supports (V = 64, K in {32, 64, 128},
 // checkpoint stride <= 16).
 bool bwd_tc_supported(int K, int V, int C);
+// Row slices (CTAs per (b, h)) of the tensor-core forward.
+int fwd_tc_slices(int B, int H, int K);
+// SMs of a B200 (the only target); used to decide when rows are sliced.
+constexpr int kNumSMs = 148;
 // Row slices (CTAs per (b, h)) of the tensor-core backward for K state rows.
 int bwd_tc_slices(int K);
 

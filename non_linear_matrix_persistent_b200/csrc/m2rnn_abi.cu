@@ -33,6 +33,7 @@ m2rnn::Params base_params(const m2rnn_dims* d, void* ws) {
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.load();
     p.dw_parts = 1;
+    p.slices = 1;
     return p;
 }
 
@@ -43,6 +44,10 @@ extern "C" {
 size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward) {
     if (check_dims(d) != M2RNN_OK) return 0;
     size_t n = kStatusBytes;
+    if (!backward && d->mode == M2RNN_MODE_BF16_TC) {   // partial readouts of sliced rows
+        const int sl = m2rnn::fwd_tc_slices(d->B, d->H, d->K);
+        if (sl > 1) n += sizeof(float) * (size_t)sl * d->B * d->H * d->T * d->V;
+    }
     if (backward) {
         const size_t extra = d->mode == M2RNN_MODE_FP32_DEBUG
                                  ? m2rnn::bwd_fp32_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride)
@@ -69,7 +74,8 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d, const void* k, const void* v, co
     const size_t state_bytes = sizeof(float) * (size_t)d->B * d->H * d->K * d->V;
     if (d->T == 0) {   // no steps: H_T = H0
         if (HT) {
-            cudaError_t e = H0 ? cudaMemcpyAsync(HT, H0, state_bytes, cudaMemcpyDeviceToDevice, s)
+            cudaError_t e = H0 ? (H0 == HT ? cudaSuccess   // in place: nothing to do
+                                           : cudaMemcpyAsync(HT, H0, state_bytes, cudaMemcpyDeviceToDevice, s))
                                : cudaMemsetAsync(HT, 0, state_bytes, s);
             if (e != cudaSuccess) return M2RNN_ERR_CUDA;
         }
@@ -77,6 +83,7 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d, const void* k, const void* v, co
     }
     m2rnn::Params p = base_params(d, workspace);
     p.k = k; p.v = v; p.q = q; p.f = f; p.W = W; p.H0 = H0; p.y = y; p.HT = HT; p.ckpt = ckpt;
+    p.ypart = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
     cudaError_t e = d->mode == M2RNN_MODE_FP32_DEBUG ? m2rnn::launch_fwd_fp32(p, s) : m2rnn::launch_fwd_tc(p, s);
     return e == cudaSuccess ? M2RNN_OK : M2RNN_ERR_CUDA;
 }
@@ -107,7 +114,8 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     }
     if (d->T == 0) {   // no steps: dH0 = dHT, dW = 0
         const size_t state_bytes = sizeof(float) * (size_t)d->B * d->H * d->K * d->V;
-        cudaError_t e = dHT ? cudaMemcpyAsync(dH0, dHT, state_bytes, cudaMemcpyDeviceToDevice, s)
+        cudaError_t e = dHT ? (dHT == dH0 ? cudaSuccess
+                                          : cudaMemcpyAsync(dH0, dHT, state_bytes, cudaMemcpyDeviceToDevice, s))
                             : cudaMemsetAsync(dH0, 0, state_bytes, s);
         if (e == cudaSuccess) e = cudaMemsetAsync(dW, 0, wbytes, s);
         return e == cudaSuccess ? M2RNN_OK : M2RNN_ERR_CUDA;

@@ -52,8 +52,8 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five workloads of the M²RNN hot path (shapes follow the pages' 410M dense
-# and 7B MoE models; see the design doc for the recipe).
+# The five workloads of the M²RNN hot path (shapes follow the 410M dense and 7B
+# MoE models of the M²RNN paper summaries; draw recipe in the module docstring).
 WORKLOADS: Dict[str, Workload] = {
     "tiny_fp32": Workload("tiny_fp32", B=1, H=1, T=64, K=16, V=16, mode="fp32"),
     "layer410m_fwd": Workload("layer410m_fwd", B=8, H=16, T=2048, K=64, V=64),

@@ -31,8 +31,11 @@ def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16):
 
 
 def test_workspace_size(L):
-    d = _dims()
-    assert L.m2rnn_workspace_size(d, 0) == 256
+    # 128 (b, h) pairs fill the GPU: one CTA per pair, the forward needs only the status word
+    assert L.m2rnn_workspace_size(_dims(B=8, H=16), 0) == 256
+    # 6 pairs: the forward splits the 64 rows into 4 slices and keeps their partial readouts
+    assert L.m2rnn_workspace_size(_dims(), 0) == 256 + 4 * (2 * 3 * 5 * 64) * 4
+    assert L.m2rnn_workspace_size(_dims(mode=1), 0) == 256   # fp32 debug mode: no slices
     assert L.m2rnn_workspace_size(_dims(mode=1), 1) > 256
     assert L.m2rnn_workspace_size(_dims(K=48), 0) == 0
     assert L.m2rnn_workspace_size(_dims(mode=7), 0) == 0

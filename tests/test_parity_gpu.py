@@ -144,6 +144,50 @@ def test_tc_batch_independence_bitwise():
     assert torch.equal(y[2:3], y1) and torch.equal(HT[2:3], HT1)
 
 
+@pytest.mark.parametrize("K", [64, 128])
+def test_row_slices_match_whole_rows(K):
+    """Few (b, h) pairs: the forward splits each pair's rows over several CTAs
+    (rows of H are independent) and sums their partial readouts.  The states
+    must equal the one-CTA-per-pair result bit for bit; y differs only in the
+    order of the readout sum."""
+    from non_linear_matrix_persistent_b200 import _lib
+    big = Workload("rs", B=8, H=16, T=37, K=K, V=64, h0_range=0.5, seed=9)
+    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(8, 16, 37, K, 64, 0, 16), 0) == 256   # one CTA per pair
+    xc = _cuda(make_inputs(big))
+    y, HT, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=8, want_ckpt=True)
+    s = {n: (None if t is None else t[3:4].contiguous()) for n, t in xc.items() if n != "W"}
+    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(1, 16, 37, K, 64, 0, 16), 0) > 256   # sliced rows
+    y1, HT1, ck1 = api().forward(s["k"], s["v"], s["q"], s["f"], xc["W"], s["H0"], ckpt_stride=8, want_ckpt=True)
+    torch.cuda.synchronize()
+    assert torch.equal(HT[3:4], HT1) and torch.equal(ck[3:4], ck1)
+    assert torch.allclose(y[3:4], y1, rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("mode,K,V", [("bf16", 64, 64), ("bf16", 128, 32), ("fp32", 32, 16)])
+def test_decode_steps_match_scan_bitwise(mode, K, V):
+    """Decode: T single-step calls that advance the state in place (H0 and H_T
+    the same buffer) give the scan's y and H_T bit for bit, and the scan
+    matches the oracle."""
+    w = Workload("dec", B=2, H=3, T=13, K=K, V=V, mode=mode, h0_range=0.5, seed=5)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    a = api()
+    y, HT, _ = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"])
+    H = xc["H0"].clone()
+    ys = []
+    for t in range(w.T):
+        col = lambda n: xc[n][:, :, t].contiguous()  # noqa: E731
+        ys.append(a.step(col("k"), col("v"), col("q"), col("f"), xc["W"], H).clone())
+    torch.cuda.synchronize()
+    assert torch.equal(torch.stack(ys, 2), y)
+    assert torch.equal(H, HT)
+    ry, rHT = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"])
+    tol = TC_ABS if mode == "bf16" else DBG_ABS
+    for got, r in ((y, ry), (HT, rHT)):
+        e_abs, _ = _errs(got, r)
+        assert e_abs <= tol
+
+
 def test_zero_steps_and_empty_batch():
     w = Workload("e", B=2, H=2, T=0, K=32, V=32, h0_range=0.5, seed=2)
     x = _cuda(make_inputs(w))
