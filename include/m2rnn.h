@@ -64,7 +64,14 @@ typedef enum {
     M2RNN_MODE_BF16_TC = 0,
     /* fp32 everything, CUDA-core FFMA and accurate tanhf: a slow reference
      * mode on the device. */
-    M2RNN_MODE_FP32_DEBUG = 1
+    M2RNN_MODE_FP32_DEBUG = 1,
+    /* As M2RNN_MODE_BF16_TC, but tanh is the single-SFU tanh.approx.f32
+     * (about 2^-11 relative error per element instead of about 1e-6
+     * absolute): a faster forward for inference, where y and H_T stay well
+     * inside the tensor-core mode's tolerance.  Forward only: m2rnn_backward
+     * returns M2RNN_ERR_INVALID_ARG and m2rnn_workspace_size(d, 1) returns 0
+     * (gradients over long sequences amplify the tanh error). */
+    M2RNN_MODE_BF16_TC_FAST_TANH = 2
 } m2rnn_mode;
 
 typedef struct {

@@ -75,10 +75,18 @@ def num_checkpoints(T: int, ckpt_stride: int) -> int:
 
 
 def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = False,
-            want_HT: bool = True, out: Optional[dict] = None):
-    """Runs the forward scan.  Returns (y, HT or None, ckpt or None)."""
+            want_HT: bool = True, out: Optional[dict] = None, fast_tanh: bool = False):
+    """Runs the forward scan.  Returns (y, HT or None, ckpt or None).
+
+    fast_tanh (bf16 inputs only) selects M2RNN_MODE_BF16_TC_FAST_TANH: the
+    single-SFU tanh.approx.f32, for inference; its checkpoints are not meant
+    for the backward, which rejects that mode."""
     dev = k.device
     d = dims_of(k, v, ckpt_stride)
+    if fast_tanh:
+        if d.mode != _lib.MODE_BF16_TC:
+            raise TypeError("fast_tanh needs bf16 inputs (the tensor-core mode)")
+        d.mode = _lib.MODE_BF16_TC_FAST_TANH
     B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
     lp = k.dtype
     _check("k", k, (B, H, T, K), lp, dev)

@@ -37,6 +37,7 @@ struct Params {
     float* dW_part;     // [B*H][dw_parts][V][V] partial dW (workspace)
     int dw_parts;       // dW partials per (b, h)
     int slices;         // forward: CTAs (row slices) per (b, h)
+    int fast_tanh;      // forward: tanh.approx.f32 instead of the exp-based tanh
     float* ypart;       // forward with slices > 1: [slices][B*H][T][V] partial readouts (workspace)
     float* scratch;     // per-CTA recompute scratch (workspace)
     uint32_t* status;   // device status word (workspace)

@@ -93,7 +93,9 @@ struct FwdTcCfg {
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
 
-template <int K, int V>
+// FAST: tanh.approx.f32 (one SFU operation, ~2^-11 relative error) instead
+// of the exp-based formula; forward-only inference mode.
+template <int K, int V, bool FAST>
 __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
     using C = FwdTcCfg<K, V>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 for (int r = 0; r < C::CH; ++r) {
                     float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
                     a = fmaf(kk[r], vj, a);
-                    const float z = tanh_exp(a);
+                    const float z = FAST ? tanh_approx(a) : tanh_exp(a);
                     h[c0 + r] = fmaf(g, z - h[c0 + r], h[c0 + r]);
                 }
             }
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
 template <int K, int V>
 static cudaError_t launch_fwd_tc_kv(const Params& p, cudaStream_t stream) {
     using C = FwdTcCfg<K, V>;
-    auto kern = m2rnn_fwd_tc_kernel<K, V>;
+    auto kern = p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true> : m2rnn_fwd_tc_kernel<K, V, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<p.B * p.H * p.slices, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);

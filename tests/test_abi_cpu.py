@@ -85,6 +85,16 @@ def test_backward_argument_errors(L):
     assert bwd(_dims(), dy=4097) == _lib.ERR_MISALIGNED
     assert bwd(_dims(mode=1), ws_bytes=256) == _lib.ERR_WORKSPACE
     assert bwd(_dims(K=8)) == _lib.ERR_UNSUPPORTED_SHAPE
+    # the fast-tanh mode is forward only
+    assert bwd(_dims(mode=_lib.MODE_BF16_TC_FAST_TANH)) == _lib.ERR_INVALID_ARG
+
+
+def test_fast_tanh_mode_workspace(L):
+    fast = _lib.MODE_BF16_TC_FAST_TANH
+    for B, H in ((2, 3), (8, 16)):
+        assert L.m2rnn_workspace_size(_dims(B=B, H=H, mode=fast), 0) == L.m2rnn_workspace_size(_dims(B=B, H=H), 0)
+    assert L.m2rnn_workspace_size(_dims(mode=fast), 1) == 0
+    assert L.m2rnn_workspace_size(_dims(mode=3), 0) == 0
 
 
 def test_status_query_rejects_null(L):

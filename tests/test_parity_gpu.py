@@ -91,6 +91,21 @@ def test_tc_forward_small(K, V, T):
     _check_fwd("tc_small_K%d_V%d_T%d" % (K, V, T), y, HT, yr, HTr, "bf16")
 
 
+@pytest.mark.parametrize("K,V", [(16, 64), (64, 64), (128, 128), (64, 16)])
+@pytest.mark.parametrize("T", [1, 40])
+def test_fast_tanh_forward_small(K, V, T):
+    """The inference mode (single-SFU tanh) against the oracle, at the
+    tensor-core tolerance."""
+    w = Workload("fast", B=2, H=3, T=T, K=K, V=V, h0_range=0.5, seed=3 * K + V + T)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], fast_tanh=True)
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    yr, HTr = _oracle_fwd(x)
+    _check_fwd("fast_small_K%d_V%d_T%d" % (K, V, T), y, HT, yr, HTr, "bf16")
+
+
 @pytest.mark.parametrize("K,V", [(16, 16), (32, 64), (64, 64), (128, 128), (64, 16)])
 @pytest.mark.parametrize("T", [1, 17, 64])
 def test_fp32_forward_small(K, V, T):
@@ -209,12 +224,13 @@ FULL = {
 }
 
 
+@pytest.mark.parametrize("fast", [False, True])
 @pytest.mark.parametrize("name", list(FULL))
-def test_full_size_forward_sampled(name):
+def test_full_size_forward_sampled(name, fast):
     w = WORKLOADS[name]
     x = make_inputs(w)
     xc = _cuda(x)
-    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"])
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], fast_tanh=fast)
     torch.cuda.synchronize()
     assert api().device_status() == 0
     assert torch.isfinite(y).all() and torch.isfinite(HT).all()
@@ -226,7 +242,7 @@ def test_full_size_forward_sampled(name):
     yr, HTr = _oracle_fwd(sel)
     ys = torch.stack([y[b, h] for b, h in pairs])[None]
     HTs = torch.stack([HT[b, h] for b, h in pairs])[None]
-    _check_fwd("full_" + name, ys, HTs, yr, HTr, "bf16")
+    _check_fwd("full_%s%s" % (name, "_fast" if fast else ""), ys, HTs, yr, HTr, "bf16")
 
 
 # ---------------------------------------------------------------- backward
