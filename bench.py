@@ -287,35 +287,69 @@ def main():
     tokens_per_step = B * T * world
     value = tokens_per_step / (ms_per_step / 1e3)
 
-    # end to end through the public API with host buffers: pinned H2D of the
-    # step's inputs, the step, D2H of its results (y and, for training, the gradients)
-    pinned = {n: (None if t is None else t.pin_memory()) for n, t in x_host.items()}
+    # End to end through the public API from host memory.  Every step copies
+    # its inputs from pinned host memory, runs the forward (and backward), and
+    # reads its results back (y and, for training, all six gradients).  Steps
+    # are pipelined as a streaming training or serving loop runs them: three
+    # streams (inputs in, compute, results out) and two device buffer sets, so
+    # that step i's compute overlaps step i+1's input copy and step i-1's
+    # result copy.  The timed region spans the first input copy to the last
+    # result copy.
+    pinned = {n: t.pin_memory() for n, t in x_host.items() if t is not None}
     res_names = ["y"] + (["dk", "dv", "dq", "df", "dW", "dH0"] if w.backward else [])
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
-    host_out = {}
-    e2e_ms = []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    nbuf = 2
+    dbuf = [{n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in pinned.items()} for _ in range(nbuf)]
+    fbuf = [{"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev),
+             "ckpt": torch.empty(B, H, (T + C - 1) // C, K, V, device=dev)} for _ in range(nbuf)]
+    gshape = {"dk": (B, H, T, K), "dv": (B, H, T, V), "dq": (B, H, T, K), "df": (B, H, T), "dW": (H, V, V),
+              "dH0": (B, H, K, V)}
+    gbuf = [{n: torch.empty(s, device=dev) for n, s in gshape.items()} for _ in range(nbuf)]
+    hbuf = [{n: torch.empty((fbuf[0]["y"] if n == "y" else gbuf[0][n]).shape, pin_memory=True) for n in res_names}
+            for _ in range(nbuf)]
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in hbuf[0].values())
+
+    def e2e_run(nsteps):
+        ev_in = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_comp = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_out = [torch.cuda.Event() for _ in range(nsteps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        xd = {n: (None if t is None else t.to(dev, non_blocking=True)) for n, t in pinned.items()}
-        y, _, ck = api.forward(xd["k"], xd["v"], xd["q"], xd["f"], xd["W"], xd["H0"], ckpt_stride=C,
-                               want_ckpt=w.backward)
-        res = {"y": y}
-        if w.backward:
-            res.update(api.backward(xd["k"], xd["v"], xd["q"], xd["f"], xd["W"], ck, xd["dY"], ckpt_stride=C))
-            parallel.allreduce_dW(res["dW"])
-        for n in res_names:
-            if n not in host_out:
-                host_out[n] = torch.empty(res[n].shape, dtype=res[n].dtype, pin_memory=True)
-            host_out[n].copy_(res[n], non_blocking=True)
-        b.record(stream)
+        t0.record(s_in)
+        for i in range(nsteps):
+            b = i % nbuf
+            with torch.cuda.stream(s_in):
+                if i >= nbuf:
+                    s_in.wait_event(ev_comp[i - nbuf])   # the compute that read this buffer set is done
+                for n, t in pinned.items():
+                    dbuf[b][n].copy_(t, non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[i])
+                if i >= nbuf:
+                    s_comp.wait_event(ev_out[i - nbuf])  # its results were read back
+                xd = dbuf[b]
+                api.forward(xd["k"], xd["v"], xd["q"], xd["f"], xd["W"], xd.get("H0"), ckpt_stride=C,
+                            want_ckpt=w.backward, out=fbuf[b])
+                if w.backward:
+                    api.backward(xd["k"], xd["v"], xd["q"], xd["f"], xd["W"], fbuf[b]["ckpt"], xd["dY"],
+                                 ckpt_stride=C, out=gbuf[b])
+                    parallel.allreduce_dW(gbuf[b]["dW"])
+                ev_comp[i].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[i])
+                for n in res_names:
+                    hbuf[b][n].copy_(fbuf[b]["y"] if n == "y" else gbuf[b][n], non_blocking=True)
+                ev_out[i].record(s_out)
+        t1.record(s_out)
         torch.cuda.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(a.elapsed_time(b))
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_total = parallel.max_over_ranks(sum(e2e_ms), dev)
+        return t0.elapsed_time(t1)
+
+    e2e_run(args.warmup)
+    if world > 1:
+        dist.barrier()
+    e2e_total = parallel.max_over_ranks(e2e_run(args.steps), dev)
     e2e_value = tokens_per_step / (e2e_total / args.steps / 1e3)
 
     peaks, peak_kind = _peaks()
@@ -358,7 +392,10 @@ def main():
                        "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
                        "l2": "flushed between timed steps (256 MB write)"},
             "clocks": clocks, "gpu_launches": launches,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_total / args.steps,
+                    "how": "pinned host inputs -> device -> fwd+bwd -> all results to pinned host, every step; "
+                           "3 streams, 2 buffer sets (step i compute overlaps i+1 copy-in and i-1 copy-out)"},
             "roofline": roofline}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
