@@ -131,16 +131,23 @@ def per_step_counts(w):
     return fwd, bwd
 
 
+def kernel_digest(src: bytes) -> str:
+    """Fingerprint of a kernel build: its source and the nvcc flags it is built with."""
+    from non_linear_matrix_persistent_b200.build import NVCC_FLAGS
+    flags = " ".join(f for f in NVCC_FLAGS if not f.startswith("-I"))
+    return hashlib.sha256(src + b"\n" + flags.encode()).hexdigest()[:16]
+
+
 def measured_traffic(kernel_file: str, profile_md: str):
     """DRAM bytes per launch recorded in a profiles/ summary, when that summary
-    was taken from the current kernel source (sha256 of the .cu file); else None."""
+    was taken from the current kernel build (kernel_digest); else None."""
     try:
         src = open(os.path.join(CSRC, kernel_file), "rb").read()
         text = open(os.path.join(ROOT, "profiles", profile_md)).read()
     except OSError:
         return None
-    digest = hashlib.sha256(src).hexdigest()[:16]
-    m = re.search(r"source sha256\[:16\] of %s: `([0-9a-f]+)`" % re.escape(kernel_file), text)
+    digest = kernel_digest(src)
+    m = re.search(r"build fingerprint of %s: `([0-9a-f]+)`" % re.escape(kernel_file), text)
     t = re.search(r"DRAM traffic per launch: ([0-9.]+) bytes", text)
     if m and t and m.group(1) == digest:
         return float(t.group(1))

