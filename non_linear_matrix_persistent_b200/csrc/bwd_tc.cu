@@ -274,18 +274,33 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // K = V = 64) is stored with L2 evict_last priority, so its round trip
         // stays in L2 instead of being written back to HBM and read again.
         const uint64_t pol_keep = l2_policy_evict_last();
+        // 32-byte accesses when the workspace allows (it is 32-byte aligned in
+        // practice; the ABI promises 16): each thread's RT values are RT·4 bytes
+        // at a multiple of RT·4
+        const bool v8 = C::RT % 8 == 0 && (reinterpret_cast<uintptr_t>(Sst) & 31) == 0;
         auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
             float* d = base + (size_t)u * K * V + tslot;
+            if (v8) {
 #pragma unroll
-            for (int g = 0; g < C::RT / 4; ++g)
-                st_global_v4_hint(d + 4 * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3], pol_keep);
+                for (int g = 0; g < C::RT / 8; ++g) st_global_v8_hint(d + 8 * g, v + 8 * g, pol_keep);
+            } else {
+#pragma unroll
+                for (int g = 0; g < C::RT / 4; ++g)
+                    st_global_v4_hint(d + 4 * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3], pol_keep);
+            }
         };
         auto ld_vec = [&](const float* base, int u, float (&v)[C::RT]) {
-            const float4* s4 = reinterpret_cast<const float4*>(base + (size_t)u * K * V + tslot);
+            const float* src = base + (size_t)u * K * V + tslot;
+            if (v8) {
 #pragma unroll
-            for (int g = 0; g < C::RT / 4; ++g) {
-                const float4 x = s4[g];
-                v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
+                for (int g = 0; g < C::RT / 8; ++g) ld_global_v8(src + 8 * g, v + 8 * g);
+            } else {
+                const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+                for (int g = 0; g < C::RT / 4; ++g) {
+                    const float4 x = s4[g];
+                    v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
+                }
             }
         };
         auto stage = [&](int i) { return smem + C::OFF_RING + (i % C::NSTAGE) * C::STAGE_BYTES; };
