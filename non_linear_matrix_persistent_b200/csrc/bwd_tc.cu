@@ -262,12 +262,16 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // chunk recomputed in phase i stores step u in slot u for even i and in
         // slot C-1-u for odd i, so in phase i+1 the recompute writes exactly
         // the slots the reverse walk (which reads its chunk from step len-1
-        // down, one step ahead) has already read.  Thread-contiguous: slot x,
-        // thread t holds its RT values at x·K·V + t·RT (16-byte vector
-        // accesses, each warp touching one contiguous block); only the thread
-        // that wrote a value reads it back.
-        float* const Sst = p.scratch + (size_t)blockIdx.x * 2 * CS * K * V;
-        float* const Sz = Sst + (size_t)CS * K * V;
+        // down, one step ahead) has already read.  Slot-major across CTAs:
+        // slot x of CTA b is the K·V block x·nCTA + b, so that the CTAs, which
+        // all touch the same slot at about the same time, hit one contiguous
+        // range instead of addresses a power of two apart (measured 2.5%
+        // faster).  Within a block, thread t holds its RT values at t·RT
+        // (each warp one contiguous run); only the thread that wrote a value
+        // reads it back.
+        const size_t nct = gridDim.x;
+        float* const Sst = p.scratch + (size_t)blockIdx.x * K * V;
+        float* const Sz = Sst + (size_t)CS * nct * K * V;
         auto sslot = [&](int i, int u) { return (i & 1) ? CS - 1 - u : u; };
         const size_t tslot = (size_t)threadIdx.x * C::RT;
         // The scratch (2·C·K·V·4 bytes per CTA, ~64 MB for 128 CTAs at C = 16,
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // at a multiple of RT·4
         const bool v8 = C::RT % 8 == 0 && (reinterpret_cast<uintptr_t>(Sst) & 31) == 0;
         auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
-            float* d = base + (size_t)u * K * V + tslot;
+            float* d = base + (size_t)u * nct * K * V + tslot;
             if (v8) {
 #pragma unroll
                 for (int g = 0; g < C::RT / 8; ++g) st_global_v8_hint(d + 8 * g, v + 8 * g, pol_keep);
@@ -290,7 +294,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
             }
         };
         auto ld_vec = [&](const float* base, int u, float (&v)[C::RT]) {
-            const float* src = base + (size_t)u * K * V + tslot;
+            const float* src = base + (size_t)u * nct * K * V + tslot;
             if (v8) {
 #pragma unroll
                 for (int g = 0; g < C::RT / 8; ++g) ld_global_v8(src + 8 * g, v + 8 * g);
