@@ -132,10 +132,16 @@ def per_step_counts(w):
 
 
 def kernel_digest(src: bytes) -> str:
-    """Fingerprint of a kernel build: its source and the nvcc flags it is built with."""
+    """Fingerprint of a kernel build: its source code (comments and blank space
+    removed, so that editing a comment keeps a profile valid) and the nvcc flags
+    it is built with."""
     from non_linear_matrix_persistent_b200.build import NVCC_FLAGS
+    text = src.decode("utf-8")
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    code = " ".join(text.split())
     flags = " ".join(f for f in NVCC_FLAGS if not f.startswith("-I"))
-    return hashlib.sha256(src + b"\n" + flags.encode()).hexdigest()[:16]
+    return hashlib.sha256((code + "\n" + flags).encode()).hexdigest()[:16]
 
 
 def measured_traffic(kernel_file: str, profile_md: str):

@@ -11,10 +11,10 @@
 //   dW   += H_{t-1}ᵀ dA_t         G_{t-1} = f_t G_t + dA_t Wᵀ,   dH0 = G_0.
 // The pages' backward recomputes the states instead of storing them (§2.2);
 // here each chunk of C steps is recomputed from the forward's checkpoint
-// H_{c·C} with exactly the forward kernel's arithmetic (same compensated
-// operand, same epilogue), so the states are bit-identical to the forward's.
-// H_{t-1} and Z_t of the chunk go to a per-CTA workspace scratch (read back
-// only by the thread that wrote them), then the chunk is walked in reverse.
+// H_{c·C} with the forward kernel's arithmetic (same compensated operand,
+// same epilogue), so the recomputed states follow the forward's.  H_{t-1}
+// and Z_t of the chunk go to a workspace scratch (read back only by the
+// thread that wrote them), then the chunk is walked in reverse.
 //
 // Layout: one CTA per (b, h) and slice of at most 64 state rows (rows of H
 // evolve independently given W, v_t and f_t), the slice's rows split into
