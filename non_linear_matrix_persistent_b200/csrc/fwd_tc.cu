@@ -6,7 +6,10 @@
 // plus the readout y_t = H_tᵀ q_t (this library's reading; the pages define
 // none).  The pages parallelise the forward over batch × head with each SM
 // owning independent matrix states (§2.2); here one CTA owns one (b, h) pair
-// for all T steps, with the fp32 state in registers.
+// for all T steps, with the fp32 state in registers.  When there are too few
+// pairs to fill the GPU, a pair's K rows are split over several CTAs (the
+// rows of H are independent given W, v_t and f_t) and the slices' partial
+// readouts are summed by m2rnn_y_reduce_kernel.
 //
 // Formulation.  The kernel computes the transpose of the transition GEMM,
 //   D = Wᵀ · H_{t-1}ᵀ   (M = V columns of H, N = state rows, contraction V),

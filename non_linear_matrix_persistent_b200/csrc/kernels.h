@@ -6,7 +6,9 @@
 
 namespace m2rnn {
 
-// tcgen05 forward scan (bf16 inputs).  K, V in {16, 32, 64, 128}.
+// tcgen05 forward scan (bf16 inputs).  K, V in {16, 32, 64, 128}; with few
+// (b, h) pairs the rows are split over fwd_tc_slices(...) CTAs per pair, and
+// the slices' partial readouts (p.ypart) are summed into y.
 cudaError_t launch_fwd_tc(const Params& p, cudaStream_t s);
 // fp32 CUDA-core forward (debug mode).
 cudaError_t launch_fwd_fp32(const Params& p, cudaStream_t s);
@@ -14,7 +16,7 @@ cudaError_t launch_fwd_fp32(const Params& p, cudaStream_t s);
 cudaError_t launch_bwd_fp32(const Params& p, cudaStream_t s);
 // tcgen05 backward (bf16 inputs): chunked recompute + BPTT + dW reduce.
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s);
-// Deterministic dW[h] = sum_b dW_part[b, h] (fixed ascending order).
+// Deterministic dW[h] = sum over b and slices of dW_part[b, h, slice] (fixed ascending order).
 cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
 
 // Shapes the tensor-core backward supports (V = 64, K in {32, 64, 128},
