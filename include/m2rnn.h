@@ -71,7 +71,15 @@ typedef enum {
      * inside the tensor-core mode's tolerance.  Forward only: m2rnn_backward
      * returns M2RNN_ERR_INVALID_ARG and m2rnn_workspace_size(d, 1) returns 0
      * (gradients over long sequences amplify the tanh error). */
-    M2RNN_MODE_BF16_TC_FAST_TANH = 2
+    M2RNN_MODE_BF16_TC_FAST_TANH = 2,
+    /* bf16 inputs, forward only, V = 64 and K in {16, 32, 64} (other shapes
+     * return M2RNN_ERR_UNSUPPORTED_SHAPE): a latency-oriented alternative
+     * forward with the state resident in registers (warp-level mma.sync, 16
+     * rows per warp, no per-step barrier).  Same compensated operand and
+     * accurate tanh as M2RNN_MODE_BF16_TC; its checkpoints may be passed to
+     * m2rnn_backward in M2RNN_MODE_BF16_TC.  m2rnn_backward rejects this mode
+     * (M2RNN_ERR_INVALID_ARG). */
+    M2RNN_MODE_BF16_MMA_SYNC = 3
 } m2rnn_mode;
 
 typedef struct {

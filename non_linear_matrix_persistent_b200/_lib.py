@@ -13,7 +13,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libm2rnn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_MISALIGNED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(7)
-MODE_BF16_TC, MODE_FP32_DEBUG, MODE_BF16_TC_FAST_TANH = 0, 1, 2
+MODE_BF16_TC, MODE_FP32_DEBUG, MODE_BF16_TC_FAST_TANH, MODE_BF16_MMA_SYNC = 0, 1, 2, 3
 
 # Every entry point declared in include/m2rnn.h.
 EXPORTS = ("m2rnn_workspace_size", "m2rnn_forward", "m2rnn_backward", "m2rnn_backward_noalloc",

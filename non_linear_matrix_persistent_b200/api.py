@@ -75,18 +75,23 @@ def num_checkpoints(T: int, ckpt_stride: int) -> int:
 
 
 def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = False,
-            want_HT: bool = True, out: Optional[dict] = None, fast_tanh: bool = False):
+            want_HT: bool = True, out: Optional[dict] = None, fast_tanh: bool = False,
+            mma_sync: bool = False):
     """Runs the forward scan.  Returns (y, HT or None, ckpt or None).
 
-    fast_tanh (bf16 inputs only) selects M2RNN_MODE_BF16_TC_FAST_TANH: the
-    single-SFU tanh.approx.f32, for inference; its checkpoints are not meant
-    for the backward, which rejects that mode."""
+    Two bf16-only alternatives to the default tensor-core forward:
+    fast_tanh selects M2RNN_MODE_BF16_TC_FAST_TANH (the single-SFU
+    tanh.approx.f32, for inference; its checkpoints are not meant for the
+    backward); mma_sync selects M2RNN_MODE_BF16_MMA_SYNC (the register-resident
+    forward for V = 64, K <= 64; its checkpoints feed the backward as usual)."""
     dev = k.device
     d = dims_of(k, v, ckpt_stride)
-    if fast_tanh:
+    if fast_tanh or mma_sync:
         if d.mode != _lib.MODE_BF16_TC:
-            raise TypeError("fast_tanh needs bf16 inputs (the tensor-core mode)")
-        d.mode = _lib.MODE_BF16_TC_FAST_TANH
+            raise TypeError("fast_tanh / mma_sync need bf16 inputs (the tensor-core mode)")
+        if fast_tanh and mma_sync:
+            raise ValueError("choose one of fast_tanh and mma_sync")
+        d.mode = _lib.MODE_BF16_TC_FAST_TANH if fast_tanh else _lib.MODE_BF16_MMA_SYNC
     B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
     lp = k.dtype
     _check("k", k, (B, H, T, K), lp, dev)

@@ -10,6 +10,9 @@ namespace m2rnn {
 // (b, h) pairs the rows are split over fwd_tc_slices(...) CTAs per pair, and
 // the slices' partial readouts (p.ypart) are summed into y.
 cudaError_t launch_fwd_tc(const Params& p, cudaStream_t s);
+// Register-resident mma.sync forward (V = 64, K in {16, 32, 64}).
+cudaError_t launch_fwd_mma(const Params& p, cudaStream_t s);
+bool fwd_mma_supported(int K, int V);
 // fp32 CUDA-core forward (debug mode).
 cudaError_t launch_fwd_fp32(const Params& p, cudaStream_t s);
 // fp32 CUDA-core backward (debug mode): chunked recompute + BPTT + dW reduce.

@@ -20,8 +20,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 m2rnn_status check_dims(const m2rnn_dims* d) {
     if (d == nullptr) return M2RNN_ERR_INVALID_ARG;
     if (d->B < 0 || d->H < 0 || d->T < 0) return M2RNN_ERR_INVALID_ARG;
-    if (d->mode != M2RNN_MODE_BF16_TC && d->mode != M2RNN_MODE_FP32_DEBUG && d->mode != M2RNN_MODE_BF16_TC_FAST_TANH)
-        return M2RNN_ERR_INVALID_ARG;
+    if (d->mode < M2RNN_MODE_BF16_TC || d->mode > M2RNN_MODE_BF16_MMA_SYNC) return M2RNN_ERR_INVALID_ARG;
     if (!shape_ok(d->K) || !shape_ok(d->V) || d->ckpt_stride < 1) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return M2RNN_OK;
 }
@@ -45,8 +44,10 @@ extern "C" {
 size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward) {
     if (check_dims(d) != M2RNN_OK) return 0;
     size_t n = kStatusBytes;
-    if (backward && d->mode == M2RNN_MODE_BF16_TC_FAST_TANH) return 0;   // forward-only mode
-    if (!backward && d->mode != M2RNN_MODE_FP32_DEBUG) {   // partial readouts of sliced rows
+    if (backward && (d->mode == M2RNN_MODE_BF16_TC_FAST_TANH || d->mode == M2RNN_MODE_BF16_MMA_SYNC))
+        return 0;   // forward-only modes
+    if (!backward && (d->mode == M2RNN_MODE_BF16_TC || d->mode == M2RNN_MODE_BF16_TC_FAST_TANH)) {
+        // partial readouts of sliced rows
         const int sl = m2rnn::fwd_tc_slices(d->B, d->H, d->K);
         if (sl > 1) n += sizeof(float) * (size_t)sl * d->B * d->H * d->T * d->V;
     }
@@ -87,7 +88,10 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d, const void* k, const void* v, co
     p.k = k; p.v = v; p.q = q; p.f = f; p.W = W; p.H0 = H0; p.y = y; p.HT = HT; p.ckpt = ckpt;
     p.ypart = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kStatusBytes);
     p.fast_tanh = d->mode == M2RNN_MODE_BF16_TC_FAST_TANH;
-    cudaError_t e = d->mode == M2RNN_MODE_FP32_DEBUG ? m2rnn::launch_fwd_fp32(p, s) : m2rnn::launch_fwd_tc(p, s);
+    cudaError_t e = d->mode == M2RNN_MODE_FP32_DEBUG    ? m2rnn::launch_fwd_fp32(p, s)
+                    : d->mode == M2RNN_MODE_BF16_MMA_SYNC ? m2rnn::launch_fwd_mma(p, s)
+                                                          : m2rnn::launch_fwd_tc(p, s);
+    if (e == cudaErrorNotSupported) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return e == cudaSuccess ? M2RNN_OK : M2RNN_ERR_CUDA;
 }
 
@@ -97,7 +101,8 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
                             m2rnn_stream_t stream) {
     m2rnn_status st = check_dims(d);
     if (st != M2RNN_OK) return st;
-    if (d->mode == M2RNN_MODE_BF16_TC_FAST_TANH) return M2RNN_ERR_INVALID_ARG;   // forward-only mode
+    if (d->mode == M2RNN_MODE_BF16_TC_FAST_TANH || d->mode == M2RNN_MODE_BF16_MMA_SYNC)
+        return M2RNN_ERR_INVALID_ARG;   // forward-only modes
     // A tensor with no elements may be passed as NULL.
     const bool seq = (long long)d->B * d->H * d->T > 0;
     const bool state = (long long)d->B * d->H > 0;

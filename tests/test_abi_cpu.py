@@ -62,7 +62,10 @@ def test_forward_argument_errors(L):
     assert _fwd(L, _dims(V=256)) == _lib.ERR_UNSUPPORTED_SHAPE
     assert _fwd(L, _dims(C=0)) == _lib.ERR_UNSUPPORTED_SHAPE
     assert _fwd(L, _dims(B=-1)) == _lib.ERR_INVALID_ARG
-    assert _fwd(L, _dims(mode=3)) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(mode=4)) == _lib.ERR_INVALID_ARG
+    # the register-resident forward covers V = 64, K <= 64 only (checked before any launch)
+    assert _fwd(L, _dims(K=128, mode=_lib.MODE_BF16_MMA_SYNC)) == _lib.ERR_UNSUPPORTED_SHAPE
+    assert _fwd(L, _dims(V=32, mode=_lib.MODE_BF16_MMA_SYNC)) == _lib.ERR_UNSUPPORTED_SHAPE
     assert _fwd(L, _dims(), {"k": None}) == _lib.ERR_INVALID_ARG
     assert _fwd(L, _dims(), {"y": None}) == _lib.ERR_INVALID_ARG
     assert _fwd(L, _dims(), {"ws": None}) == _lib.ERR_INVALID_ARG
@@ -85,8 +88,9 @@ def test_backward_argument_errors(L):
     assert bwd(_dims(), dy=4097) == _lib.ERR_MISALIGNED
     assert bwd(_dims(mode=1), ws_bytes=256) == _lib.ERR_WORKSPACE
     assert bwd(_dims(K=8)) == _lib.ERR_UNSUPPORTED_SHAPE
-    # the fast-tanh mode is forward only
+    # the fast-tanh and register-resident modes are forward only
     assert bwd(_dims(mode=_lib.MODE_BF16_TC_FAST_TANH)) == _lib.ERR_INVALID_ARG
+    assert bwd(_dims(mode=_lib.MODE_BF16_MMA_SYNC)) == _lib.ERR_INVALID_ARG
 
 
 def test_fast_tanh_mode_workspace(L):
@@ -94,7 +98,13 @@ def test_fast_tanh_mode_workspace(L):
     for B, H in ((2, 3), (8, 16)):
         assert L.m2rnn_workspace_size(_dims(B=B, H=H, mode=fast), 0) == L.m2rnn_workspace_size(_dims(B=B, H=H), 0)
     assert L.m2rnn_workspace_size(_dims(mode=fast), 1) == 0
-    assert L.m2rnn_workspace_size(_dims(mode=3), 0) == 0
+    assert L.m2rnn_workspace_size(_dims(mode=4), 0) == 0
+
+
+def test_mma_sync_mode_workspace(L):
+    mma = _lib.MODE_BF16_MMA_SYNC
+    assert L.m2rnn_workspace_size(_dims(mode=mma), 0) == 256   # one CTA per pair, no slices
+    assert L.m2rnn_workspace_size(_dims(mode=mma), 1) == 0     # forward only
 
 
 def test_status_query_rejects_null(L):

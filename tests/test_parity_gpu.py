@@ -106,6 +106,51 @@ def test_fast_tanh_forward_small(K, V, T):
     _check_fwd("fast_small_K%d_V%d_T%d" % (K, V, T), y, HT, yr, HTr, "bf16")
 
 
+@pytest.mark.parametrize("K", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 17, 40])
+def test_mma_sync_forward_small(K, T):
+    """The register-resident forward against the oracle, at the tensor-core tolerance."""
+    w = Workload("mma", B=2, H=3, T=T, K=K, V=64, h0_range=0.5, seed=5 * K + T)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], mma_sync=True)
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    yr, HTr = _oracle_fwd(x)
+    _check_fwd("mma_small_K%d_T%d" % (K, T), y, HT, yr, HTr, "bf16")
+
+
+def test_mma_sync_forward_full_size_and_checkpoints_feed_backward():
+    """At the 410M layer shape, sampled pairs against the oracle; and the
+    register-resident forward's checkpoints drive the tensor-core backward."""
+    a = api()
+    w = WORKLOADS["layer410m_fwd"]
+    x = make_inputs(w)
+    xc = _cuda(x)
+    y, HT, _ = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], mma_sync=True)
+    torch.cuda.synchronize()
+    pairs = FULL["layer410m_fwd"]
+    yr, HTr = _oracle_fwd(_select_pairs(x, pairs))
+    _check_fwd("full_layer410m_fwd_mma", torch.stack([y[b, h] for b, h in pairs])[None],
+               torch.stack([HT[b, h] for b, h in pairs])[None], yr, HTr, "bf16")
+    wt = Workload("mmabwd", B=2, H=2, T=37, K=64, V=64, h0_range=0.5, backward=True, seed=4)
+    xt = make_inputs(wt)
+    xtc = _cuda(xt)
+    _, _, ck = a.forward(xtc["k"], xtc["v"], xtc["q"], xtc["f"], xtc["W"], xtc["H0"], ckpt_stride=8,
+                         want_ckpt=True, mma_sync=True)
+    g = a.backward(xtc["k"], xtc["v"], xtc["q"], xtc["f"], xtc["W"], ck, xtc["dY"], ckpt_stride=8)
+    torch.cuda.synchronize()
+    _check_grads("mma_ckpt_backward", g, _oracle_bwd(xt), GRAD_REL)
+
+
+def test_mma_sync_unsupported_shape():
+    from non_linear_matrix_persistent_b200._lib import M2RNNError
+    w = Workload("mmax", B=1, H=1, T=4, K=128, V=64, seed=1)
+    xc = _cuda(make_inputs(w))
+    with pytest.raises(M2RNNError):
+        api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], mma_sync=True)
+
+
 @pytest.mark.parametrize("K,V", [(16, 16), (32, 64), (64, 64), (128, 128), (64, 16)])
 @pytest.mark.parametrize("T", [1, 17, 64])
 def test_fp32_forward_small(K, V, T):
