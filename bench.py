@@ -185,6 +185,13 @@ def _oracle_sample(w, pairs, cores):
     return run
 
 
+def bench_config(w, world):
+    """The workload description both arms print (same keys, same values)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "K": w.K, "V": w.V, "ckpt_stride": CKPT_STRIDE,
+            "global_batch": w.B * world, "seq_len": w.T, "parallelism": "dp%d" % world,
+            "l2": "flushed between timed steps (256 MB write)"}
+
+
 def run_reference(args, w):
     """fp64 CPU oracle on a bounded sample of (b, h) pairs at full length."""
     from oracle import oracle
@@ -204,7 +211,7 @@ def run_reference(args, w):
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "K": w.K, "V": w.V},
+            "data": "synthetic", "config": bench_config(w, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -401,9 +408,7 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": B, "H": H, "T": T, "K": K, "V": V, "ckpt_stride": C,
-                       "global_batch": B * world, "seq_len": T, "parallelism": "dp%d" % world,
-                       "l2": "flushed between timed steps (256 MB write)"},
+            "config": bench_config(w, world),
             "clocks": clocks, "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_total / args.steps,
