@@ -7,7 +7,7 @@ import importlib
 
 from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
 
-_API_NAMES = ("forward", "backward", "device_status", "set_wait_limit_ns")
+_API_NAMES = ("forward", "backward", "step", "device_status", "set_wait_limit_ns")
 
 
 def __getattr__(name):

@@ -5,10 +5,12 @@ device memory and the current stream.  Names follow include/m2rnn.h.
 
   y, HT, ckpt = forward(k, v, q, f, W, H0=None, ckpt_stride=16, want_ckpt=False)
   grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=16)
+  y_t         = step(k_t, v_t, q_t, f_t, W, H)        # one decode step, H updated in place
 
 bf16 k/v/q/W select the tensor-core mode (M2RNN_MODE_BF16_TC); fp32 select
-the fp32 debug mode.  Tensors must be contiguous CUDA tensors with the
-head-first layouts of the header.
+the fp32 debug mode; forward(..., fast_tanh=True) and forward(...,
+mma_sync=True) select the forward-only alternatives.  Tensors must be
+contiguous CUDA tensors with the head-first layouts of the header.
 """
 from __future__ import annotations
 
