@@ -121,3 +121,21 @@ def test_binding_signatures_match_header(L):
         assert m, name
         params = [x for x in m.group(1).split(",") if x.strip() and x.strip() != "void"]
         assert len(getattr(L, name).argtypes) == len(params), (name, len(params))
+
+
+def test_api_mode_flags_are_checked_before_any_launch():
+    import torch
+    from non_linear_matrix_persistent_b200 import api
+    B, H, T, K, V = 1, 1, 2, 16, 16
+    f32 = dict(dtype=torch.float32)
+    k, q = torch.zeros(B, H, T, K, **f32), torch.zeros(B, H, T, K, **f32)
+    v, f, W = torch.zeros(B, H, T, V, **f32), torch.zeros(B, H, T, **f32), torch.zeros(H, V, V, **f32)
+    with pytest.raises(TypeError):          # the alternatives need bf16 inputs
+        api.forward(k, v, q, f, W, fast_tanh=True)
+    with pytest.raises(TypeError):
+        api.forward(k, v, q, f, W, mma_sync=True)
+    bf = [t.to(torch.bfloat16) for t in (k, v, q)]
+    with pytest.raises(ValueError):         # one alternative at a time
+        api.forward(bf[0], bf[1], bf[2], f, W.to(torch.bfloat16), fast_tanh=True, mma_sync=True)
+    with pytest.raises(ValueError):         # step needs the state buffer
+        api.step(k[:, :, 0], v[:, :, 0], q[:, :, 0], f[:, :, 0], W, None)
