@@ -77,9 +77,24 @@ def default_threads() -> int:
     return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
 
 
+def _heads_of_groups(a: np.ndarray, H: int) -> np.ndarray:
+    """Grouped-value form (gist.science technical summary §2.2, tensor
+    parallelism: the topology-aware strategy keeps a group's heads together;
+    the other strategy all-reduces the gradients of the query and key that
+    heads share).  Reading: k and q carry G head groups, G dividing H, and
+    head h uses the k and q of group h // (H / G); v, f, W and the state stay
+    per head.  Returns the per-head [B, H, T, K] view of a [B, G, T, K] array."""
+    G = a.shape[1]
+    assert G >= 1 and H % G == 0, (G, H)
+    return a if G == H else np.repeat(a, H // G, axis=1)
+
+
 def forward(k, v, q, f, W, H0=None, nthreads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
-    """Returns (y [B,H,T,V], H_T [B,H,K,V]) in fp64."""
+    """Returns (y [B,H,T,V], H_T [B,H,K,V]) in fp64.  k and q may be
+    [B,G,T,K] with G dividing H (grouped-value form, _heads_of_groups)."""
     k, v, q, f, W, H0 = (_f64(a) for a in (k, v, q, f, W, H0))
+    H = v.shape[1]
+    k, q = _heads_of_groups(k, H), _heads_of_groups(q, H)
     B, H, T, K = k.shape
     V = v.shape[-1]
     assert v.shape == (B, H, T, V) and q.shape == (B, H, T, K) and f.shape == (B, H, T)
@@ -94,8 +109,14 @@ def forward(k, v, q, f, W, H0=None, nthreads: Optional[int] = None) -> Tuple[np.
 
 
 def backward(k, v, q, f, W, H0, dy, dHT=None, nthreads: Optional[int] = None):
-    """Returns dict of fp64 gradients dk, dv, dq, df, dW, dH0 for loss with dL/dy = dy, dL/dH_T = dHT."""
+    """Returns dict of fp64 gradients dk, dv, dq, df, dW, dH0 for loss with dL/dy = dy, dL/dH_T = dHT.
+
+    With grouped k and q ([B,G,T,K], _heads_of_groups) dk and dq are [B,G,T,K]:
+    the gradient of a shared input is the sum of its uses' gradients, here
+    over the H / G heads of the group."""
     k, v, q, f, W, H0, dy, dHT = (_f64(a) for a in (k, v, q, f, W, H0, dy, dHT))
+    G, H = k.shape[1], v.shape[1]
+    k, q = _heads_of_groups(k, H), _heads_of_groups(q, H)
     B, H, T, K = k.shape
     V = v.shape[-1]
     assert dy.shape == (B, H, T, V) and (dHT is None or dHT.shape == (B, H, K, V))
@@ -107,4 +128,7 @@ def backward(k, v, q, f, W, H0, dy, dHT=None, nthreads: Optional[int] = None):
         _ptr(out["dH0"]), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("oracle backward failed (%d)" % rc)
+    if G != H:
+        for n in ("dk", "dq"):
+            out[n] = out[n].reshape(B, G, H // G, T, K).sum(axis=2)
     return out

@@ -291,3 +291,75 @@ def test_backward_closed_form_W0_f0():
     np.testing.assert_allclose(g["df"], (G * (Hprev - Z)).sum((-1, -2)), rtol=0, atol=1e-12)
     np.testing.assert_allclose(g["dW"], np.einsum("bhtil,bhtij->hlj", Hprev, dA), rtol=0, atol=1e-12)
     np.testing.assert_array_equal(g["dH0"], np.zeros_like(H0))
+
+
+# ---------------------------------------------------------------- grouped q / k
+# Grouped-value form (gist.science technical summary §2.2, tensor parallelism):
+# k and q carry G groups of heads, head h uses group h // (H / G).
+
+def _grouped(B=2, H=4, G=2, T=5, K=3, V=2, seed=21):
+    k, v, q, f, W, H0 = _rand(B=B, H=H, T=T, K=K, V=V, seed=seed)
+    r = np.random.default_rng(seed + 1)
+    kg = r.standard_normal((B, G, T, K)) * 0.7
+    qg = r.standard_normal((B, G, T, K)) * 0.7
+    return kg, v, qg, f, W, H0
+
+
+def test_grouped_heads_read_their_own_group():
+    # Changing the k (or q) of group g changes exactly the heads g·H/G .. (g+1)·H/G - 1,
+    # which pins the head -> group map (consecutive heads share, not h mod G).
+    k, v, q, f, W, H0 = _grouped(H=6, G=3)
+    y0, HT0 = oracle.forward(k, v, q, f, W, H0)
+    for name in ("k", "q"):
+        for g in range(3):
+            k2, q2 = k.copy(), q.copy()
+            (k2 if name == "k" else q2)[:, g] += 0.3
+            y1, HT1 = oracle.forward(k2, v, q2, f, W, H0)
+            changed = [h for h in range(6) if not np.array_equal(y1[:, h], y0[:, h])]
+            assert changed == [2 * g, 2 * g + 1], (name, g, changed)
+            if name == "q":   # q only enters the readout
+                np.testing.assert_array_equal(HT1, HT0)
+
+
+def test_one_group_with_equal_heads_gives_equal_heads():
+    # G = 1 and every head given the same v, f, W, H0: all heads see the same
+    # recurrence, so their outputs are bitwise equal; dk, dq are then H times
+    # the gradient of one head with its own (ungrouped) k and q.
+    k, v, q, f, W, H0 = _grouped(H=3, G=1)
+    v[:] = v[:, :1]; f[:] = f[:, :1]; W[:] = W[:1]; H0[:] = H0[:, :1]
+    y, HT = oracle.forward(k, v, q, f, W, H0)
+    for h in range(1, 3):
+        np.testing.assert_array_equal(y[:, h], y[:, 0])
+        np.testing.assert_array_equal(HT[:, h], HT[:, 0])
+    r = np.random.default_rng(22)
+    dy1 = r.standard_normal(v[:, :1].shape)
+    dy = np.repeat(dy1, 3, axis=1)
+    g = oracle.backward(k, v, q, f, W, H0, dy)
+    g1 = oracle.backward(k, v[:, :1], q, f[:, :1], W[:1], H0[:, :1], dy1)
+    np.testing.assert_allclose(g["dk"], 3 * g1["dk"], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(g["dq"], 3 * g1["dq"], rtol=1e-13, atol=1e-15)
+
+
+def test_grouped_backward_finite_differences():
+    k, v, q, f, W, H0 = _grouped(H=4, G=2)
+    r = np.random.default_rng(23)
+    dy = r.standard_normal(v.shape)
+    dHT = r.standard_normal(H0.shape)
+    g = oracle.backward(k, v, q, f, W, H0, dy, dHT, nthreads=1)
+    assert g["dk"].shape == k.shape and g["dq"].shape == q.shape
+    args = {"k": k, "v": v, "q": q, "f": f, "W": W, "H0": H0}
+    names = {"k": "dk", "v": "dv", "q": "dq", "f": "df", "W": "dW", "H0": "dH0"}
+    eps = 1e-6
+    for name, arr in args.items():
+        flat = arr.reshape(-1)
+        idx = r.choice(flat.size, size=min(flat.size, 10), replace=False)
+        for e in idx:
+            old = flat[e]
+            flat[e] = old + eps
+            lp = _loss(dy=dy, dHT=dHT, **args)
+            flat[e] = old - eps
+            lm = _loss(dy=dy, dHT=dHT, **args)
+            flat[e] = old
+            fd = (lp - lm) / (2 * eps)
+            an = g[names[name]].reshape(-1)[e]
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (name, e, fd, an)
