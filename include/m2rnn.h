@@ -16,9 +16,16 @@
  * this library's reading: the pages define no readout.
  *
  * Layout: every tensor is dense, contiguous, head-first, row-major:
- *   k, q   [B][H][T][K]      v, y, dy   [B][H][T][V]      f, df  [B][H][T]
+ *   k, q, dk, dq   [B][G][T][K]      v, y, dy   [B][H][T][V]      f, df  [B][H][T]
  *   W, dW  [H][V][V]         H0, HT, dHT, dH0  [B][H][K][V]
  *   ckpt   [B][H][ceil(T/C)][K][V]   (C = ckpt_stride; ckpt[.,.,c] = H_{c·C})
+ * G = H unless k and q are grouped (m2rnn_dims.qk_heads): G groups of H/G
+ * consecutive heads, head h reading the k and q of group h / (H/G), while
+ * v, f, W and the state stay per head.  This is the library's reading of the
+ * grouped-value form of the pages' tensor-parallel scheme (gist.science
+ * §2.2: the topology-aware strategy needs no communication; the other one
+ * all-reduces the gradients of the query and key that heads share).  dk and
+ * dq of a group are the sums over its heads, in ascending head order.
  * Element types: in M2RNN_MODE_BF16_TC the inputs k, v, q, W, dy are bf16
  * (raw 16-bit words) and everything else is fp32.  In M2RNN_MODE_FP32_DEBUG
  * all tensors are fp32.
@@ -48,7 +55,7 @@ extern "C" {
 
 typedef enum {
     M2RNN_OK = 0,
-    M2RNN_ERR_INVALID_ARG = 1,       /* NULL required pointer, negative size, bad mode */
+    M2RNN_ERR_INVALID_ARG = 1,       /* NULL required pointer, negative size, bad mode or qk_heads */
     M2RNN_ERR_UNSUPPORTED_SHAPE = 2, /* K or V outside {16,32,64,128}, ckpt_stride < 1 */
     M2RNN_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
     M2RNN_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than m2rnn_workspace_size */
@@ -86,6 +93,9 @@ typedef struct {
     int B, H, T, K, V;  /* batch, heads, steps, state rows (key dim), state columns (value dim) */
     int mode;           /* m2rnn_mode */
     int ckpt_stride;    /* C >= 1: the forward stores H_{c·C} for the backward */
+    int qk_heads;       /* G, the head groups of k and q: 0 (or H) = one per head;
+                         * otherwise 1 <= G < H with H % G == 0, else
+                         * M2RNN_ERR_INVALID_ARG */
 } m2rnn_dims;
 
 /* Same type as cudaStream_t; NULL is the legacy default stream. */
@@ -95,7 +105,9 @@ typedef struct CUstream_st* m2rnn_stream_t;
  * Returns 0 for invalid dims.  The first 256 bytes hold the device status
  * word: zero them once after allocating the workspace.  The rest is scratch
  * the kernels write before they read it: for the backward, per-(b, h) dW
- * partials and the chunk recompute buffer; for a tensor-core forward with
+ * partials and the chunk recompute buffer, plus, when k and q are grouped,
+ * the per-head dk and dq (2 · B·H·T·K fp32) summed into the groups' dk and
+ * dq at the end; for a tensor-core forward with
  * few (b, h) pairs (B·H·2 <= 148), which splits each pair's K rows over
  * several CTAs, the slices' partial readouts (slices · B·H·T·V fp32). */
 size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward);

@@ -7,6 +7,9 @@ device memory and the current stream.  Names follow include/m2rnn.h.
   grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=16)
   y_t         = step(k_t, v_t, q_t, f_t, W, H)        # one decode step, H updated in place
 
+k and q may carry fewer heads than v (G dividing H: grouped k / q, head h
+uses group h // (H // G)); dk and dq then have G heads too.
+
 bf16 k/v/q/W select the tensor-core mode (M2RNN_MODE_BF16_TC); fp32 select
 the fp32 debug mode; forward(..., fast_tanh=True) and forward(...,
 mma_sync=True) select the forward-only alternatives.  Tensors must be
@@ -55,8 +58,13 @@ def _check(name, t, shape, dtype, device):
 
 
 def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16) -> Dims:
-    B, H, T, K = k.shape
-    return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride)
+    """Dims of a call: H from v, the k / q head groups G from k."""
+    B, G, T, K = k.shape
+    H = v.shape[1]
+    if G < 1 or H % G != 0:
+        if H > 0 or G > 0:
+            raise ValueError("k has %d heads: it must have H = %d heads or a divisor of H" % (G, H))
+    return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride, G if G != H else 0)
 
 
 def workspace(d: Dims, backward: bool, device) -> torch.Tensor:
@@ -96,9 +104,10 @@ def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = 
         d.mode = _lib.MODE_BF16_TC_FAST_TANH if fast_tanh else _lib.MODE_BF16_MMA_SYNC
     B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
     lp = k.dtype
-    _check("k", k, (B, H, T, K), lp, dev)
+    G = d.qk_heads or H
+    _check("k", k, (B, G, T, K), lp, dev)
     _check("v", v, (B, H, T, V), lp, dev)
-    _check("q", q, (B, H, T, K), lp, dev)
+    _check("q", q, (B, G, T, K), lp, dev)
     _check("f", f, (B, H, T), torch.float32, dev)
     _check("W", W, (H, V, V), lp, dev)
     _check("H0", H0, (B, H, K, V), torch.float32, dev)
@@ -122,12 +131,12 @@ def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = 
 
 def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None):
     """One decode step, in place: advances the fp32 state H [B, H, K, V] by one
-    step of the recurrence with k, q [B, H, K], v [B, H, V] and f [B, H], and
-    returns y [B, H, V].  It is the forward with T = 1 and the state buffer
-    passed as both H0 and H_T (the ABI allows that alias), so T calls give the
-    scan's outputs bit for bit."""
-    B, Hh, K = k.shape
-    V = v.shape[-1]
+    step of the recurrence with k, q [B, H, K] (or [B, G, K], grouped), v
+    [B, H, V] and f [B, H], and returns y [B, H, V].  It is the forward with
+    T = 1 and the state buffer passed as both H0 and H_T (the ABI allows that
+    alias), so T calls give the scan's outputs bit for bit."""
+    B, _, K = k.shape
+    Hh, V = v.shape[1], v.shape[-1]
     if H is None:
         raise ValueError("step needs the state buffer H (it is updated in place)")
     _check("H", H, (B, Hh, K, V), torch.float32, k.device)
@@ -144,16 +153,17 @@ def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: O
     d = dims_of(k, v, ckpt_stride)
     B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
     lp = k.dtype
-    _check("k", k, (B, H, T, K), lp, dev)
+    G = d.qk_heads or H
+    _check("k", k, (B, G, T, K), lp, dev)
     _check("v", v, (B, H, T, V), lp, dev)
-    _check("q", q, (B, H, T, K), lp, dev)
+    _check("q", q, (B, G, T, K), lp, dev)
     _check("f", f, (B, H, T), torch.float32, dev)
     _check("W", W, (H, V, V), lp, dev)
     _check("ckpt", ckpt, (B, H, num_checkpoints(T, ckpt_stride), K, V), torch.float32, dev)
     _check("dy", dy, (B, H, T, V), lp, dev)
     _check("dHT", dHT, (B, H, K, V), torch.float32, dev)
     out = dict(out or {})
-    shapes = {"dk": (B, H, T, K), "dv": (B, H, T, V), "dq": (B, H, T, K), "df": (B, H, T),
+    shapes = {"dk": (B, G, T, K), "dv": (B, H, T, V), "dq": (B, G, T, K), "df": (B, H, T),
               "dW": (H, V, V), "dH0": (B, H, K, V)}
     for n, s in shapes.items():
         if out.get(n) is None:

@@ -532,6 +532,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer (chunks in reverse order)
         int last = -1, last_ck = -1;   // last chunk whose inputs / checkpoint were requested
+        const int qkb = qk_pair(p, bh);   // k / q rows of this pair's head group
         for (int i = 0; i < nck; ++i) {
             const int c0 = (nck - 1 - i) * CS, len = min(CS, T - c0), s = i % C::NSTAGE;
             if (i >= C::NSTAGE) {
@@ -547,7 +548,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 // dy rows c0-1 .. c0+len-1; the row of step c0-1 exists only when c0 > 0
                 const uint32_t dyb = (uint32_t)((len + (c0 > 0 ? 1 : 0)) * V * 2);
                 mbar_arrive_expect_tx(in_full(s), 2 * kb + vb + dyb);
-                const size_t rk = ((size_t)bh * T + c0) * KF, rv = ((size_t)bh * T + c0) * V;
+                const size_t rk = ((size_t)qkb * T + c0) * KF, rv = ((size_t)bh * T + c0) * V;
                 const uint16_t* dyg = static_cast<const uint16_t*>(p.dy) + rv;
                 bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + rk, kb, in_full(s));
                 bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + rk, kb, in_full(s));

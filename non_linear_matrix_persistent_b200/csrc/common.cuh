@@ -16,6 +16,7 @@ enum : uint32_t {
 
 struct Params {
     int B, H, T, K, V, C;
+    int G;              // head groups of k and q (G divides H; G == H: one per head)
     const void* k;
     const void* v;
     const void* q;
@@ -44,6 +45,12 @@ struct Params {
     uint64_t wait_limit_ns;
     int fault;          // injected fault (m2rnn_debug_set_fault), 0 = none
 };
+
+// Row block of k and q that pair bh = b·H + h reads: head h uses group
+// h / (H/G) of batch element b.  The identity when G == H.
+__host__ __device__ __forceinline__ int qk_pair(const Params& p, int bh) {
+    return (bh / p.H) * p.G + (bh % p.H) / (p.H / p.G);
+}
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA-wide
 // abort flag and the device status word) when the wait runs longer than the

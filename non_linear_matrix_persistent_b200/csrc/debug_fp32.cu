@@ -53,8 +53,9 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_fwd_fp32_kernel(const Param
     const float* kg = static_cast<const float*>(p.k);
     const float* vg = static_cast<const float*>(p.v);
     const float* qg = static_cast<const float*>(p.q);
+    const size_t qkb = (size_t)qk_pair(p, bh);   // k / q rows of this pair's head group
     for (int t = 0; t < T; ++t) {
-        const size_t rk = ((size_t)bh * T + t) * K, rv = ((size_t)bh * T + t) * V;
+        const size_t rk = (qkb * T + t) * K, rv = ((size_t)bh * T + t) * V;
         for (int i = threadIdx.x; i < K; i += blockDim.x) { kt[i] = kg[rk + i]; qt[i] = qg[rk + i]; }
         for (int j = threadIdx.x; j < V; j += blockDim.x) vt[j] = vg[rv + j];
         const float ft = p.f[(size_t)bh * T + t];
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
     const float* vg = static_cast<const float*>(p.v);
     const float* qg = static_cast<const float*>(p.q);
     const float* dyg = static_cast<const float*>(p.dy);
+    const size_t qkb = (size_t)qk_pair(p, bh);   // k / q rows of this pair's head group
     __syncthreads();
     for (int c = nck - 1; c >= 0; --c) {
         const int c0 = c * C, len = min(C, T - c0);
@@ -119,8 +121,8 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
         __syncthreads();
         for (int u = 0; u < len; ++u) {   // recompute the chunk's states
             const int t = c0 + u;
-            const size_t rk = ((size_t)bh * T + t) * K, rv = ((size_t)bh * T + t) * V;
-            for (int i = threadIdx.x; i < K; i += blockDim.x) kt[i] = kg[rk + i];
+            const size_t rq = (qkb * T + t) * K, rv = ((size_t)bh * T + t) * V;
+            for (int i = threadIdx.x; i < K; i += blockDim.x) kt[i] = kg[rq + i];
             for (int j = threadIdx.x; j < V; j += blockDim.x) vt[j] = vg[rv + j];
             __syncthreads();
             dbg_step(K, V, S + (size_t)u * K * V, Ws, kt, vt, p.f[(size_t)bh * T + t], S + (size_t)(u + 1) * K * V);
@@ -130,8 +132,9 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
             const int t = c0 + u;
             const float* Hp = S + (size_t)u * K * V;
             const float* Hn = S + (size_t)(u + 1) * K * V;
-            const size_t rk = ((size_t)bh * T + t) * K, rv = ((size_t)bh * T + t) * V;
-            for (int i = threadIdx.x; i < K; i += blockDim.x) { kt[i] = kg[rk + i]; qt[i] = qg[rk + i]; }
+            // rk: this pair's row of dk / dq (per head; summed over a head group afterwards)
+            const size_t rk = ((size_t)bh * T + t) * K, rq = (qkb * T + t) * K, rv = ((size_t)bh * T + t) * V;
+            for (int i = threadIdx.x; i < K; i += blockDim.x) { kt[i] = kg[rq + i]; qt[i] = qg[rq + i]; }
             for (int j = threadIdx.x; j < V; j += blockDim.x) { vt[j] = vg[rv + j]; dyt[j] = dyg[rv + j]; }
             const float ft = p.f[(size_t)bh * T + t];
             __syncthreads();

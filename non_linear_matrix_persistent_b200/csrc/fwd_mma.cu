@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
         if (ok && p.HT != nullptr) store_state(p.HT + sbase);
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer
+        const int qkb = qk_pair(p, bh);   // k / q rows of this pair's head group
         int last = -1;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % C::S;
@@ -231,9 +232,9 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
             if (lane == 0) {
                 const uint32_t kb = (uint32_t)(nt * K * 2), vb = (uint32_t)(nt * V * 2);
                 mbar_arrive_expect_tx(in_full(s), 2 * kb + vb);
-                bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + ((size_t)bh * T + t0) * K, kb,
+                bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + ((size_t)qkb * T + t0) * K, kb,
                          in_full(s));
-                bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + ((size_t)bh * T + t0) * K, kb,
+                bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + ((size_t)qkb * T + t0) * K, kb,
                          in_full(s));
                 bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + ((size_t)bh * T + t0) * V, vb,
                          in_full(s));

@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
         }
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer
+        const int qkb = qk_pair(p, bh);   // k / q rows of this pair's head group
         int last = -1;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % C::S;
@@ -285,9 +286,9 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 const uint32_t kb = (uint32_t)(nt * K * 2), vb = (uint32_t)(nt * V * 2);
                 mbar_arrive_expect_tx(in_full(s), 2 * kb + vb);
                 if (nsl == 1) {
-                    bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + ((size_t)bh * T + t0) * K, kb,
+                    bulk_g2s(smem_u32(st + C::ST_K), static_cast<const uint16_t*>(p.k) + ((size_t)qkb * T + t0) * K, kb,
                              in_full(s));
-                    bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + ((size_t)bh * T + t0) * K, kb,
+                    bulk_g2s(smem_u32(st + C::ST_Q), static_cast<const uint16_t*>(p.q) + ((size_t)qkb * T + t0) * K, kb,
                              in_full(s));
                 }
                 bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + ((size_t)bh * T + t0) * V, vb,
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 // this slice's K values of each step's k and q row (strided in HBM)
                 __syncwarp();
                 if (lane < nt) {
-                    const size_t r = ((size_t)bh * T + t0 + lane) * KF + koff;
+                    const size_t r = ((size_t)qkb * T + t0 + lane) * KF + koff;
                     bulk_g2s(smem_u32(st + C::ST_K + lane * K * 2), static_cast<const uint16_t*>(p.k) + r, K * 2,
                              in_full(s));
                     bulk_g2s(smem_u32(st + C::ST_Q + lane * K * 2), static_cast<const uint16_t*>(p.q) + r, K * 2,

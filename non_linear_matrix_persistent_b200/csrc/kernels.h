@@ -21,6 +21,10 @@ cudaError_t launch_bwd_fp32(const Params& p, cudaStream_t s);
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s);
 // Deterministic dW[h] = sum over b and slices of dW_part[b, h, slice] (fixed ascending order).
 cudaError_t launch_dw_reduce(const Params& p, cudaStream_t s);
+// Grouped k / q: dk, dq [B, G, T, K] = sums over each group's heads of the
+// per-head dk_part, dq_part [B, H, T, K] (ascending head order).
+cudaError_t launch_qk_group_reduce(const Params& p, const float* dk_part, const float* dq_part, float* dk, float* dq,
+                                   cudaStream_t s);
 
 // Shapes the tensor-core backward supports (V = 64, K in {32, 64, 128},
 // checkpoint stride <= 16).

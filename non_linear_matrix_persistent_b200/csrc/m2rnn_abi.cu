@@ -21,14 +21,27 @@ m2rnn_status check_dims(const m2rnn_dims* d) {
     if (d == nullptr) return M2RNN_ERR_INVALID_ARG;
     if (d->B < 0 || d->H < 0 || d->T < 0) return M2RNN_ERR_INVALID_ARG;
     if (d->mode < M2RNN_MODE_BF16_TC || d->mode > M2RNN_MODE_BF16_MMA_SYNC) return M2RNN_ERR_INVALID_ARG;
+    // k / q head groups: 0 = one per head, else a divisor of H
+    if (d->qk_heads < 0 || (d->qk_heads > 0 && (d->qk_heads > d->H || d->H % d->qk_heads != 0)))
+        return M2RNN_ERR_INVALID_ARG;
     if (!shape_ok(d->K) || !shape_ok(d->V) || d->ckpt_stride < 1) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return M2RNN_OK;
+}
+
+int qk_groups(const m2rnn_dims* d) { return d->qk_heads > 0 ? d->qk_heads : d->H; }
+
+// Backward with grouped k / q: per-head dk and dq (fp32 [B][H][T][K] each)
+// before the sum over each group's heads.
+size_t qk_group_partial_bytes(const m2rnn_dims* d) {
+    if (qk_groups(d) == d->H) return 0;
+    return 2 * sizeof(float) * (size_t)d->B * d->H * d->T * d->K;
 }
 
 m2rnn::Params base_params(const m2rnn_dims* d, void* ws) {
     m2rnn::Params p;
     std::memset(&p, 0, sizeof p);
     p.B = d->B; p.H = d->H; p.T = d->T; p.K = d->K; p.V = d->V; p.C = d->ckpt_stride;
+    p.G = qk_groups(d);
     p.status = static_cast<uint32_t*>(ws);
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.load();
@@ -56,6 +69,7 @@ size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward) {
                                  ? m2rnn::bwd_fp32_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride)
                                  : m2rnn::bwd_tc_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride);
         n += (extra + 255) / 256 * 256;
+        n += qk_group_partial_bytes(d);
     }
     return n;
 }
@@ -136,7 +150,16 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     p.dW_part = reinterpret_cast<float*>(extra);
     p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K);
     p.scratch = p.dW_part + (size_t)d->B * d->H * p.dw_parts * d->V * d->V;
+    const bool grouped = qk_group_partial_bytes(d) != 0;
+    if (grouped) {   // the kernels write per-head dk / dq here; the group sums go to dk, dq
+        const size_t extra_bytes = d->mode == M2RNN_MODE_FP32_DEBUG
+                                       ? m2rnn::bwd_fp32_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride)
+                                       : m2rnn::bwd_tc_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride);
+        p.dk = reinterpret_cast<float*>(extra + (extra_bytes + 255) / 256 * 256);
+        p.dq = p.dk + (size_t)d->B * d->H * d->T * d->K;
+    }
     cudaError_t e = d->mode == M2RNN_MODE_FP32_DEBUG ? m2rnn::launch_bwd_fp32(p, s) : m2rnn::launch_bwd_tc(p, s);
+    if (e == cudaSuccess && grouped) e = m2rnn::launch_qk_group_reduce(p, p.dk, p.dq, dk, dq, s);
     if (e == cudaErrorNotSupported) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return e == cudaSuccess ? M2RNN_OK : M2RNN_ERR_CUDA;
 }

@@ -15,8 +15,9 @@ Draw recipe (one torch CPU ``Generator`` seeded once, draws in this order):
   (round-to-nearest-even, torch's cast).  f, H0 stay fp32.
 
 Tensors are head-first and contiguous:
-  k, q [B, H, T, K]; v [B, H, T, V]; f [B, H, T]; W [H, V, V];
+  k, q [B, G, T, K]; v [B, H, T, V]; f [B, H, T]; W [H, V, V];
   H0 [B, H, K, V]; dY [B, H, T, V].
+G = H unless ``qk_heads`` is set (k and q shared by groups of H / G heads).
 """
 from __future__ import annotations
 
@@ -43,6 +44,7 @@ class Workload:
     h0_range: float = 0.0       # 0 -> H0 = 0, else U(-h0_range, h0_range)
     backward: bool = False      # whether the workload includes BPTT
     seed: int = 0
+    qk_heads: int = 0           # k / q head groups G (0: one per head)
 
     @property
     def tokens(self) -> int:
@@ -74,9 +76,10 @@ def make_inputs(w: Workload, device: Optional[str] = None) -> Dict[str, torch.Te
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
     B, H, T, K, V = w.B, w.H, w.T, w.K, w.V
-    k = torch.randn(B, H, T, K, generator=g) * (1.0 / math.sqrt(K))
+    G = w.qk_heads or H
+    k = torch.randn(B, G, T, K, generator=g) * (1.0 / math.sqrt(K))
     v = torch.randn(B, H, T, V, generator=g) * (1.0 / math.sqrt(V))
-    q = torch.randn(B, H, T, K, generator=g) * (1.0 / math.sqrt(K))
+    q = torch.randn(B, G, T, K, generator=g) * (1.0 / math.sqrt(K))
     z = torch.randn(B, H, T, generator=g) * math.sqrt(w.gate_var)
     f = torch.sigmoid(z + w.gate_shift)
     W = torch.randn(H, V, V, generator=g) * (1.0 / math.sqrt(V))

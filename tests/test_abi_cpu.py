@@ -26,8 +26,8 @@ def test_exports_match_header(L):
         assert hasattr(L, name), name
 
 
-def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16):
-    return _lib.Dims(B, H, T, K, V, mode, C)
+def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16, G=0):
+    return _lib.Dims(B, H, T, K, V, mode, C, G)
 
 
 def test_workspace_size(L):
@@ -105,6 +105,36 @@ def test_mma_sync_mode_workspace(L):
     mma = _lib.MODE_BF16_MMA_SYNC
     assert L.m2rnn_workspace_size(_dims(mode=mma), 0) == 256   # one CTA per pair, no slices
     assert L.m2rnn_workspace_size(_dims(mode=mma), 1) == 0     # forward only
+
+
+def test_grouped_qk_heads(L):
+    """k / q head groups: 0 or H = one per head; otherwise a proper divisor of
+    H.  The backward keeps per-head dk and dq (2·B·H·T·K fp32) before summing
+    each group; the forward needs nothing extra."""
+    for mode in (0, 1):
+        for B, H in ((2, 4), (8, 16)):
+            plain = [L.m2rnn_workspace_size(_dims(B=B, H=H, mode=mode), bw) for bw in (0, 1)]
+            assert [L.m2rnn_workspace_size(_dims(B=B, H=H, mode=mode, G=H), bw) for bw in (0, 1)] == plain
+            for G in (1, 2):
+                d = _dims(B=B, H=H, mode=mode, G=G)
+                assert L.m2rnn_workspace_size(d, 0) == plain[0]
+                assert L.m2rnn_workspace_size(d, 1) == plain[1] + 2 * B * H * 5 * 64 * 4
+    for G in (-1, 2, 4):   # negative, not a divisor of H = 3, more groups than heads
+        assert L.m2rnn_workspace_size(_dims(G=G), 0) == 0
+        assert _fwd(L, _dims(G=G)) == _lib.ERR_INVALID_ARG
+    assert _fwd(L, _dims(B=0, H=0, G=1)) == _lib.ERR_INVALID_ARG
+
+
+def test_api_grouped_shapes_are_checked_on_the_host():
+    import torch
+    from non_linear_matrix_persistent_b200 import api
+    B, H, T, K, V = 1, 4, 2, 16, 16
+    bf = dict(dtype=torch.bfloat16)
+    v = torch.zeros(B, H, T, V, **bf)
+    assert api.dims_of(torch.zeros(B, 2, T, K, **bf), v).qk_heads == 2
+    assert api.dims_of(torch.zeros(B, 4, T, K, **bf), v).qk_heads == 0   # one per head
+    with pytest.raises(ValueError):
+        api.dims_of(torch.zeros(B, 3, T, K, **bf), v)
 
 
 def test_status_query_rejects_null(L):

@@ -370,3 +370,75 @@ def test_train_workload_sampled_head():
     gr = _oracle_bwd(sel)
     gs = {n: (t[:, h:h + 1] if n != "dW" else t[h:h + 1]) for n, t in g.items()}
     _check_grads("full_layer410m_train_head%d" % h, gs, gr, GRAD_REL)
+
+
+# ---------------------------------------------------------------- grouped k / q
+# k and q with G < H head groups (head h reads group h // (H / G)); dk and dq
+# are the sums over each group's heads.  B·H = 128 pairs run one CTA per pair,
+# fewer pairs split rows over several CTAs (and K = 128 backward over two).
+
+GROUPED = [(2, 4, 2, 64), (2, 4, 1, 128), (1, 6, 3, 32), (8, 16, 4, 64)]
+
+
+@pytest.mark.parametrize("B,H,G,K", GROUPED)
+@pytest.mark.parametrize("variant", ["tc", "fast", "mma", "fp32"])
+def test_grouped_forward(B, H, G, K, variant):
+    if variant == "mma" and K > 64:
+        pytest.skip("the register-resident forward covers K <= 64")
+    mode = "fp32" if variant == "fp32" else "bf16"
+    w = Workload("gq", B=B, H=H, T=21, K=K, V=64, mode=mode, h0_range=0.5, qk_heads=G, seed=G + K + H)
+    x = make_inputs(w)
+    assert x["k"].shape[1] == G and x["q"].shape[1] == G
+    xc = _cuda(x)
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"],
+                             fast_tanh=variant == "fast", mma_sync=variant == "mma")
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    yr, HTr = _oracle_fwd(x)
+    _check_fwd("grouped_fwd_%s_B%d_H%d_G%d_K%d" % (variant, B, H, G, K), y, HT, yr, HTr, mode)
+
+
+@pytest.mark.parametrize("B,H,G,K", GROUPED)
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+@pytest.mark.parametrize("T,C", [(1, 16), (37, 8)])
+def test_grouped_backward(B, H, G, K, mode, T, C):
+    w = Workload("gqb", B=B, H=H, T=T, K=K, V=64, mode=mode, h0_range=0.5, backward=True, qk_heads=G,
+                 seed=3 * G + K + T)
+    x = make_inputs(w)
+    dHT = torch.randn(B, H, K, 64, generator=torch.Generator().manual_seed(5))
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, C, dHT.cuda())
+    assert g["dk"].shape == (B, G, T, K) and g["dq"].shape == (B, G, T, K)
+    gr = _oracle_bwd(x, dHT)
+    _check_grads("grouped_bwd_%s_B%d_H%d_G%d_K%d_T%d" % (mode, B, H, G, K, T), g, gr,
+                 GRAD_REL if mode == "bf16" else 1e-4)
+
+
+@pytest.mark.parametrize("B,H,G,K", [(2, 4, 2, 64), (8, 16, 4, 64), (2, 4, 1, 128)])
+def test_grouped_equals_repeated_inputs_bitwise(B, H, G, K):
+    """A grouped call computes exactly what the ungrouped call computes on k
+    and q repeated over each group's heads: y, H_T, dv, df, dW and dH0 bit for
+    bit, and dk, dq equal to the ascending-head sums of the per-head results."""
+    w = Workload("gqr", B=B, H=H, T=29, K=K, V=64, h0_range=0.5, backward=True, qk_heads=G, seed=G * K)
+    xc = _cuda(make_inputs(w))
+    rep = dict(xc)
+    for n in ("k", "q"):
+        rep[n] = xc[n].repeat_interleave(H // G, dim=1).contiguous()
+    a = api()
+    outs = []
+    for x in (xc, rep):
+        y, HT, ck = a.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=8, want_ckpt=True)
+        g = a.backward(x["k"], x["v"], x["q"], x["f"], x["W"], ck, x["dY"], ckpt_stride=8)
+        outs.append((y.clone(), HT.clone(), {n: t.clone() for n, t in g.items()}))
+    torch.cuda.synchronize()
+    assert a.device_status() == 0
+    (y, HT, g), (yr, HTr, gr) = outs
+    assert torch.equal(y, yr) and torch.equal(HT, HTr)
+    for n in ("dv", "df", "dW", "dH0"):
+        assert torch.equal(g[n], gr[n]), n
+    for n in ("dk", "dq"):
+        per = gr[n].view(B, G, H // G, 29, K)
+        s = per[:, :, 0].clone()
+        for j in range(1, H // G):
+            s = s + per[:, :, j]
+        assert torch.equal(g[n], s), n
