@@ -59,3 +59,49 @@ def test_two_rank_dW_allreduce_matches_global_batch(tmp_path):
         np.testing.assert_allclose(res["dW"], g["dW"], rtol=1e-12, atol=1e-12)
         np.testing.assert_array_equal(res["dk"], g["dk"][r * W0.B:(r + 1) * W0.B])
         assert float(res["t_max"]) == float(world)
+
+
+# ---------------------------------------------------------------- heads sharded
+# Topology-aware tensor parallelism: each rank holds whole k / q head groups and
+# their heads; nothing is exchanged, and the ranks' results are slices of the
+# single-process result.
+
+W_TP = Workload("tp", B=2, H=4, T=7, K=4, V=6, h0_range=0.5, backward=True, qk_heads=2, seed=8)
+
+
+def _tp_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    from non_linear_matrix_persistent_b200 import make_inputs, parallel
+    from oracle import oracle
+    r, ws = parallel.init("gloo", timeout_s=60)
+    x = parallel.head_shard(make_inputs(W_TP), r, ws)
+    y, HT = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], nthreads=1)
+    g = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], nthreads=1)
+    np.savez(os.path.join(out_dir, "tp%d.npz" % r), y=y, HT=HT, **g)
+    import torch.distributed as dist
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_head_shards_need_no_exchange(tmp_path):
+    from non_linear_matrix_persistent_b200 import make_inputs
+    from oracle import oracle
+    world = 2
+    mp.start_processes(_tp_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    x = make_inputs(W_TP)
+    y, HT = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], nthreads=1)
+    g = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], nthreads=1)
+    res = [np.load(os.path.join(str(tmp_path), "tp%d.npz" % r)) for r in range(world)]
+    for n, ref in dict(y=y, HT=HT, dv=g["dv"], df=g["df"], dH0=g["dH0"], dk=g["dk"], dq=g["dq"]).items():
+        np.testing.assert_array_equal(np.concatenate([r[n] for r in res], axis=1), ref, err_msg=n)
+    np.testing.assert_array_equal(np.concatenate([r["dW"] for r in res], axis=0), g["dW"])
+
+
+def test_head_shard_rejects_uneven_groups():
+    from non_linear_matrix_persistent_b200 import make_inputs, parallel
+    x = make_inputs(W_TP.with_(qk_heads=0, H=3, backward=False))
+    with pytest.raises(ValueError):
+        parallel.head_shard(x, 0, 2)
+    s = parallel.head_shard(make_inputs(W_TP), 1, 2)
+    assert s["k"].shape[1] == 1 and s["v"].shape[1] == 2 and s["W"].shape[0] == 2
