@@ -89,10 +89,25 @@ def _heads_of_groups(a: np.ndarray, H: int) -> np.ndarray:
     return a if G == H else np.repeat(a, H // G, axis=1)
 
 
-def forward(k, v, q, f, W, H0=None, nthreads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+def gate_from_logit(a: np.ndarray) -> np.ndarray:
+    """Forget gate from a gate logit (gist.science technical summary §2.1: a
+    parameterised ψ(x_t) keeps f_t in [0, 1], with per-head decay rates at
+    initialisation).  Reading: ψ ends in the logistic function,
+    f_t = 1 / (1 + exp(-a_t)); how a_t is computed from x_t (a projection and
+    a per-head bias that sets each head's initial decay) lies outside the
+    recurrence, so a_t is an input."""
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-a))
+
+
+def forward(k, v, q, f, W, H0=None, nthreads: Optional[int] = None,
+            f_is_logit: bool = False) -> Tuple[np.ndarray, np.ndarray]:
     """Returns (y [B,H,T,V], H_T [B,H,K,V]) in fp64.  k and q may be
-    [B,G,T,K] with G dividing H (grouped-value form, _heads_of_groups)."""
+    [B,G,T,K] with G dividing H (grouped-value form, _heads_of_groups).  With
+    f_is_logit, f holds gate logits a_t and f_t = gate_from_logit(a_t)."""
     k, v, q, f, W, H0 = (_f64(a) for a in (k, v, q, f, W, H0))
+    if f_is_logit:
+        f = gate_from_logit(f)
     H = v.shape[1]
     k, q = _heads_of_groups(k, H), _heads_of_groups(q, H)
     B, H, T, K = k.shape
@@ -108,13 +123,17 @@ def forward(k, v, q, f, W, H0=None, nthreads: Optional[int] = None) -> Tuple[np.
     return y, HT
 
 
-def backward(k, v, q, f, W, H0, dy, dHT=None, nthreads: Optional[int] = None):
+def backward(k, v, q, f, W, H0, dy, dHT=None, nthreads: Optional[int] = None, f_is_logit: bool = False):
     """Returns dict of fp64 gradients dk, dv, dq, df, dW, dH0 for loss with dL/dy = dy, dL/dH_T = dHT.
 
     With grouped k and q ([B,G,T,K], _heads_of_groups) dk and dq are [B,G,T,K]:
     the gradient of a shared input is the sum of its uses' gradients, here
-    over the H / G heads of the group."""
+    over the H / G heads of the group.  With f_is_logit, f holds gate logits
+    a_t (see forward) and df is dL/da_t = dL/df_t · f_t (1 - f_t), the chain
+    rule through the logistic function."""
     k, v, q, f, W, H0, dy, dHT = (_f64(a) for a in (k, v, q, f, W, H0, dy, dHT))
+    if f_is_logit:
+        f = gate_from_logit(f)
     G, H = k.shape[1], v.shape[1]
     k, q = _heads_of_groups(k, H), _heads_of_groups(q, H)
     B, H, T, K = k.shape
@@ -131,4 +150,6 @@ def backward(k, v, q, f, W, H0, dy, dHT=None, nthreads: Optional[int] = None):
     if G != H:
         for n in ("dk", "dq"):
             out[n] = out[n].reshape(B, G, H // G, T, K).sum(axis=2)
+    if f_is_logit:
+        out["df"] = out["df"] * f * (1.0 - f)
     return out

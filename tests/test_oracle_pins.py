@@ -363,3 +363,51 @@ def test_grouped_backward_finite_differences():
             fd = (lp - lm) / (2 * eps)
             an = g[names[name]].reshape(-1)[e]
             assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (name, e, fd, an)
+
+
+# ---------------------------------------------------------------- gate logits
+# f_t = 1 / (1 + exp(-a_t)) from a gate logit a_t (reading of the forget gate's
+# parameterisation ψ, gist.science technical summary §2.1).
+
+def test_gate_logit_values():
+    a = np.array([0.0, np.log(3.0), -np.log(3.0), 50.0, -800.0])
+    np.testing.assert_allclose(oracle.gate_from_logit(a), [0.5, 0.75, 0.25, 1.0, 0.0], rtol=1e-15, atol=1e-300)
+
+
+def test_gate_logit_forward_is_the_forward_of_the_gate_value():
+    # a = log(f / (1 - f)) inverts the logistic: the logit path must reproduce
+    # the value path (a flipped sign would give the gate 1 - f instead)
+    k, v, q, f, W, H0 = _rand(seed=31)
+    a = np.log(f / (1.0 - f))
+    y, HT = oracle.forward(k, v, q, f, W, H0)
+    ya, HTa = oracle.forward(k, v, q, a, W, H0, f_is_logit=True)
+    np.testing.assert_allclose(ya, y, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(HTa, HT, rtol=0, atol=1e-13)
+    # a saturated logit is f = 1 exactly: the state stays H0
+    _, HT1 = oracle.forward(k, v, q, np.full_like(f, 50.0), W, H0, f_is_logit=True)
+    np.testing.assert_array_equal(HT1, H0)
+
+
+def test_gate_logit_backward_finite_differences():
+    k, v, q, f, W, H0 = _rand(B=2, H=2, T=6, K=3, V=4, seed=33)
+    a = np.random.default_rng(34).standard_normal(f.shape) * 2.0
+    r = np.random.default_rng(35)
+    dy = r.standard_normal(v.shape)
+    dHT = r.standard_normal(H0.shape)
+    g = oracle.backward(k, v, q, a, W, H0, dy, dHT, nthreads=1, f_is_logit=True)
+    eps = 1e-6
+    flat = a.reshape(-1)
+    for e in range(flat.size):
+        old = flat[e]
+        flat[e] = old + eps
+        yp, HTp = oracle.forward(k, v, q, a, W, H0, nthreads=1, f_is_logit=True)
+        flat[e] = old - eps
+        ym, HTm = oracle.forward(k, v, q, a, W, H0, nthreads=1, f_is_logit=True)
+        flat[e] = old
+        fd = (((yp - ym) * dy).sum() + ((HTp - HTm) * dHT).sum()) / (2 * eps)
+        an = g["df"].reshape(-1)[e]
+        assert abs(fd - an) <= 1e-7 * max(1.0, abs(fd)), (e, fd, an)
+    # the other gradients do not depend on how f was given
+    gv = oracle.backward(k, v, q, oracle.gate_from_logit(a), W, H0, dy, dHT, nthreads=1)
+    for n in ("dk", "dv", "dq", "dW", "dH0"):
+        np.testing.assert_array_equal(g[n], gv[n])
