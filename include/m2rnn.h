@@ -55,7 +55,7 @@ extern "C" {
 
 typedef enum {
     M2RNN_OK = 0,
-    M2RNN_ERR_INVALID_ARG = 1,       /* NULL required pointer, negative size, bad mode or qk_heads */
+    M2RNN_ERR_INVALID_ARG = 1,       /* NULL required pointer, negative size, bad mode, qk_heads or f_is_logit */
     M2RNN_ERR_UNSUPPORTED_SHAPE = 2, /* K or V outside {16,32,64,128}, ckpt_stride < 1 */
     M2RNN_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
     M2RNN_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than m2rnn_workspace_size */
@@ -96,6 +96,15 @@ typedef struct {
     int qk_heads;       /* G, the head groups of k and q: 0 (or H) = one per head;
                          * otherwise 1 <= G < H with H % G == 0, else
                          * M2RNN_ERR_INVALID_ARG */
+    int f_is_logit;     /* 0: f holds the gate f_t in [0, 1].  1: f holds gate
+                         * logits a_t and f_t = 1 / (1 + exp(-a_t)), evaluated
+                         * in the kernels (accurate expf); m2rnn_backward then
+                         * writes dL/da_t = dL/df_t · f_t (1 - f_t) to df.
+                         * Other values: M2RNN_ERR_INVALID_ARG.  The library's
+                         * reading of the gate parameterisation ψ(x_t) (gist.science
+                         * §2.1 forget gate): ψ ends in the logistic function;
+                         * how a_t comes from x_t (a projection, a per-head bias
+                         * setting each head's initial decay) is the caller's. */
 } m2rnn_dims;
 
 /* Same type as cudaStream_t; NULL is the legacy default stream. */

@@ -24,7 +24,7 @@ EXPORTS = ("m2rnn_workspace_size", "m2rnn_forward", "m2rnn_backward", "m2rnn_bac
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("K", ctypes.c_int),
                 ("V", ctypes.c_int), ("mode", ctypes.c_int), ("ckpt_stride", ctypes.c_int),
-                ("qk_heads", ctypes.c_int)]
+                ("qk_heads", ctypes.c_int), ("f_is_logit", ctypes.c_int)]
 
 
 class M2RNNError(RuntimeError):

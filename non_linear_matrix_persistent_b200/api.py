@@ -8,7 +8,9 @@ device memory and the current stream.  Names follow include/m2rnn.h.
   y_t         = step(k_t, v_t, q_t, f_t, W, H)        # one decode step, H updated in place
 
 k and q may carry fewer heads than v (G dividing H: grouped k / q, head h
-uses group h // (H // G)); dk and dq then have G heads too.
+uses group h // (H // G)); dk and dq then have G heads too.  With
+f_is_logit=True, f holds gate logits a_t (f_t = sigmoid(a_t), evaluated in
+the kernels) and backward returns dL/da_t as df.
 
 bf16 k/v/q/W select the tensor-core mode (M2RNN_MODE_BF16_TC); fp32 select
 the fp32 debug mode; forward(..., fast_tanh=True) and forward(...,
@@ -57,14 +59,14 @@ def _check(name, t, shape, dtype, device):
         raise ValueError("%s must be contiguous" % name)
 
 
-def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16) -> Dims:
+def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16, f_is_logit: bool = False) -> Dims:
     """Dims of a call: H from v, the k / q head groups G from k."""
     B, G, T, K = k.shape
     H = v.shape[1]
     if G < 1 or H % G != 0:
         if H > 0 or G > 0:
             raise ValueError("k has %d heads: it must have H = %d heads or a divisor of H" % (G, H))
-    return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride, G if G != H else 0)
+    return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride, G if G != H else 0, int(bool(f_is_logit)))
 
 
 def workspace(d: Dims, backward: bool, device) -> torch.Tensor:
@@ -86,7 +88,7 @@ def num_checkpoints(T: int, ckpt_stride: int) -> int:
 
 def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = False,
             want_HT: bool = True, out: Optional[dict] = None, fast_tanh: bool = False,
-            mma_sync: bool = False):
+            mma_sync: bool = False, f_is_logit: bool = False):
     """Runs the forward scan.  Returns (y, HT or None, ckpt or None).
 
     Two bf16-only alternatives to the default tensor-core forward:
@@ -95,7 +97,7 @@ def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = 
     backward); mma_sync selects M2RNN_MODE_BF16_MMA_SYNC (the register-resident
     forward for V = 64, K <= 64; its checkpoints feed the backward as usual)."""
     dev = k.device
-    d = dims_of(k, v, ckpt_stride)
+    d = dims_of(k, v, ckpt_stride, f_is_logit)
     if fast_tanh or mma_sync:
         if d.mode != _lib.MODE_BF16_TC:
             raise TypeError("fast_tanh / mma_sync need bf16 inputs (the tensor-core mode)")
@@ -129,7 +131,7 @@ def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = 
     return y, HT, ckpt
 
 
-def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None):
+def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None, f_is_logit: bool = False):
     """One decode step, in place: advances the fp32 state H [B, H, K, V] by one
     step of the recurrence with k, q [B, H, K] (or [B, G, K], grouped), v
     [B, H, V] and f [B, H], and returns y [B, H, V].  It is the forward with
@@ -143,14 +145,15 @@ def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None):
     if y is None:
         y = torch.empty(B, Hh, V, dtype=torch.float32, device=k.device)
     forward(k.unsqueeze(2), v.unsqueeze(2), q.unsqueeze(2), f.unsqueeze(2), W, H, ckpt_stride=1,
-            out={"y": y.view(B, Hh, 1, V), "HT": H})
+            out={"y": y.view(B, Hh, 1, V), "HT": H}, f_is_logit=f_is_logit)
     return y
 
 
-def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: Optional[dict] = None):
+def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: Optional[dict] = None,
+             f_is_logit: bool = False):
     """BPTT from the forward's checkpoints.  Returns dict dk, dv, dq, df, dW, dH0 (fp32)."""
     dev = k.device
-    d = dims_of(k, v, ckpt_stride)
+    d = dims_of(k, v, ckpt_stride, f_is_logit)
     B, H, T, K, V = d.B, d.H, d.T, d.K, d.V
     lp = k.dtype
     G = d.qk_heads or H

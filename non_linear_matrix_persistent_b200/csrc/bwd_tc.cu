@@ -541,7 +541,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 if (!ok) break;
             }
             uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
-            if (lane < len) reinterpret_cast<float*>(st + C::ST_F)[lane] = p.f[(size_t)bh * T + c0 + lane];
+            if (lane < len)
+                reinterpret_cast<float*>(st + C::ST_F)[lane] = gate_value(p, p.f[(size_t)bh * T + c0 + lane]);
             __syncwarp();
             if (lane == 0) {
                 const uint32_t kb = (uint32_t)(len * KF * 2), vb = (uint32_t)(len * V * 2);
@@ -691,6 +692,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 float sf = 0.f;
 #pragma unroll
                 for (int w = 0; w < C::NWE; ++w) sf += part[C::DFP / 4 + lane * C::NWE + w];
+                sf = gate_grad(p, p.f[(size_t)bh * T + c0 + lane], sf);   // per slice: the chain rule is linear
                 float* dst = p.df + (size_t)bh * T + c0 + lane;
                 if constexpr (NSL == 1) *dst = sf;
                 else atomicAdd(dst, sf);

@@ -17,6 +17,7 @@ enum : uint32_t {
 struct Params {
     int B, H, T, K, V, C;
     int G;              // head groups of k and q (G divides H; G == H: one per head)
+    int f_is_logit;     // f holds gate logits a_t, f_t = 1 / (1 + exp(-a_t)); df is then dL/da_t
     const void* k;
     const void* v;
     const void* q;
@@ -50,6 +51,19 @@ struct Params {
 // h / (H/G) of batch element b.  The identity when G == H.
 __host__ __device__ __forceinline__ int qk_pair(const Params& p, int bh) {
     return (bh / p.H) * p.G + (bh % p.H) / (p.H / p.G);
+}
+
+// Gate f_t from the f input: the value itself, or the logistic function of a
+// gate logit (accurate expf and IEEE division; saturates to exactly 0 or 1).
+__device__ __forceinline__ float gate_value(const Params& p, float x) {
+    return p.f_is_logit ? 1.f / (1.f + expf(-x)) : x;
+}
+
+// dL/df_t -> the gradient of the f input: unchanged, or dL/da_t = dL/df_t · f_t (1 - f_t).
+__device__ __forceinline__ float gate_grad(const Params& p, float x, float df) {
+    if (!p.f_is_logit) return df;
+    const float ft = gate_value(p, x);
+    return df * (ft * (1.f - ft));
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA-wide

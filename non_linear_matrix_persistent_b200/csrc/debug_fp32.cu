@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_fwd_fp32_kernel(const Param
         const size_t rk = (qkb * T + t) * K, rv = ((size_t)bh * T + t) * V;
         for (int i = threadIdx.x; i < K; i += blockDim.x) { kt[i] = kg[rk + i]; qt[i] = qg[rk + i]; }
         for (int j = threadIdx.x; j < V; j += blockDim.x) vt[j] = vg[rv + j];
-        const float ft = p.f[(size_t)bh * T + t];
+        const float ft = gate_value(p, p.f[(size_t)bh * T + t]);
         __syncthreads();
         dbg_step(K, V, Hc, Ws, kt, vt, ft, Hn);
         __syncthreads();
@@ -125,7 +125,8 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
             for (int i = threadIdx.x; i < K; i += blockDim.x) kt[i] = kg[rq + i];
             for (int j = threadIdx.x; j < V; j += blockDim.x) vt[j] = vg[rv + j];
             __syncthreads();
-            dbg_step(K, V, S + (size_t)u * K * V, Ws, kt, vt, p.f[(size_t)bh * T + t], S + (size_t)(u + 1) * K * V);
+            dbg_step(K, V, S + (size_t)u * K * V, Ws, kt, vt, gate_value(p, p.f[(size_t)bh * T + t]),
+                     S + (size_t)(u + 1) * K * V);
             __syncthreads();
         }
         for (int u = len - 1; u >= 0; --u) {
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
             const size_t rk = ((size_t)bh * T + t) * K, rq = (qkb * T + t) * K, rv = ((size_t)bh * T + t) * V;
             for (int i = threadIdx.x; i < K; i += blockDim.x) { kt[i] = kg[rq + i]; qt[i] = qg[rq + i]; }
             for (int j = threadIdx.x; j < V; j += blockDim.x) { vt[j] = vg[rv + j]; dyt[j] = dyg[rv + j]; }
-            const float ft = p.f[(size_t)bh * T + t];
+            const float ft = gate_value(p, p.f[(size_t)bh * T + t]);
             __syncthreads();
             for (int e = threadIdx.x; e < K * V; e += blockDim.x) G[e] = fmaf(qt[e / V], dyt[e % V], G[e]);
             __syncthreads();
@@ -150,7 +151,7 @@ __global__ void __launch_bounds__(kDbgThreads) m2rnn_bwd_fp32_kernel(const Param
                 dA[e] = (1.f - ft) * G[e] * (1.f - z * z);
             }
             const float dfs = block_sum(dfp, red);
-            if (threadIdx.x == 0) p.df[(size_t)bh * T + t] = dfs;
+            if (threadIdx.x == 0) p.df[(size_t)bh * T + t] = gate_grad(p, p.f[(size_t)bh * T + t], dfs);
             __syncthreads();
             for (int i = threadIdx.x; i < K; i += blockDim.x) {
                 float s = 0.f, s2 = 0.f;

@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
             }
             const int t0 = c * C::TC, nt = min(C::TC, T - t0);
             uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
-            if (lane < nt) reinterpret_cast<float*>(st + C::ST_F)[lane] = p.f[(size_t)bh * T + t0 + lane];
+            if (lane < nt)
+                reinterpret_cast<float*>(st + C::ST_F)[lane] = gate_value(p, p.f[(size_t)bh * T + t0 + lane]);
             __syncwarp();
             if (lane == 0) {
                 const uint32_t kb = (uint32_t)(nt * K * 2), vb = (uint32_t)(nt * V * 2);

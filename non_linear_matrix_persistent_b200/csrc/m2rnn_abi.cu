@@ -24,6 +24,7 @@ m2rnn_status check_dims(const m2rnn_dims* d) {
     // k / q head groups: 0 = one per head, else a divisor of H
     if (d->qk_heads < 0 || (d->qk_heads > 0 && (d->qk_heads > d->H || d->H % d->qk_heads != 0)))
         return M2RNN_ERR_INVALID_ARG;
+    if (d->f_is_logit != 0 && d->f_is_logit != 1) return M2RNN_ERR_INVALID_ARG;
     if (!shape_ok(d->K) || !shape_ok(d->V) || d->ckpt_stride < 1) return M2RNN_ERR_UNSUPPORTED_SHAPE;
     return M2RNN_OK;
 }
@@ -42,6 +43,7 @@ m2rnn::Params base_params(const m2rnn_dims* d, void* ws) {
     std::memset(&p, 0, sizeof p);
     p.B = d->B; p.H = d->H; p.T = d->T; p.K = d->K; p.V = d->V; p.C = d->ckpt_stride;
     p.G = qk_groups(d);
+    p.f_is_logit = d->f_is_logit;
     p.status = static_cast<uint32_t*>(ws);
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.fault = g_fault.load();

@@ -10,6 +10,8 @@ Draw recipe (one torch CPU ``Generator`` seeded once, draws in this order):
   W ~ N(0, 1/V) per head, dY ~ N(0, 1).
 * The gate value is ``f = sigmoid(z + shift)`` with ``z ~ N(0, gate_var)``; it is
   an input here (the gate parameterisation psi(x_t) is outside the recurrence).
+  With ``gate_logits`` the workload passes the logit ``z + shift`` instead (the
+  kernels then apply the logistic function).
 * H0 is zero, or U(-h0_range, h0_range) when ``h0_range > 0``.
 * All draws are fp32; in bf16 mode k, v, q, W and dY are then rounded to bf16
   (round-to-nearest-even, torch's cast).  f, H0 stay fp32.
@@ -45,6 +47,7 @@ class Workload:
     backward: bool = False      # whether the workload includes BPTT
     seed: int = 0
     qk_heads: int = 0           # k / q head groups G (0: one per head)
+    gate_logits: bool = False   # f holds the gate logit z + gate_shift instead of its sigmoid
 
     @property
     def tokens(self) -> int:
@@ -81,7 +84,7 @@ def make_inputs(w: Workload, device: Optional[str] = None) -> Dict[str, torch.Te
     v = torch.randn(B, H, T, V, generator=g) * (1.0 / math.sqrt(V))
     q = torch.randn(B, G, T, K, generator=g) * (1.0 / math.sqrt(K))
     z = torch.randn(B, H, T, generator=g) * math.sqrt(w.gate_var)
-    f = torch.sigmoid(z + w.gate_shift)
+    f = (z + w.gate_shift) if w.gate_logits else torch.sigmoid(z + w.gate_shift)
     W = torch.randn(H, V, V, generator=g) * (1.0 / math.sqrt(V))
     H0 = None
     if w.h0_range > 0:

@@ -26,8 +26,8 @@ def test_exports_match_header(L):
         assert hasattr(L, name), name
 
 
-def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16, G=0):
-    return _lib.Dims(B, H, T, K, V, mode, C, G)
+def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16, G=0, logit=0):
+    return _lib.Dims(B, H, T, K, V, mode, C, G, logit)
 
 
 def test_workspace_size(L):
@@ -135,6 +135,15 @@ def test_api_grouped_shapes_are_checked_on_the_host():
     assert api.dims_of(torch.zeros(B, 4, T, K, **bf), v).qk_heads == 0   # one per head
     with pytest.raises(ValueError):
         api.dims_of(torch.zeros(B, 3, T, K, **bf), v)
+
+
+def test_gate_logit_flag(L):
+    for mode in (0, 1):
+        for bw in (0, 1):
+            assert L.m2rnn_workspace_size(_dims(mode=mode, logit=1), bw) == L.m2rnn_workspace_size(_dims(mode=mode), bw)
+    for bad in (-1, 2):
+        assert L.m2rnn_workspace_size(_dims(logit=bad), 0) == 0
+        assert _fwd(L, _dims(logit=bad)) == _lib.ERR_INVALID_ARG
 
 
 def test_status_query_rejects_null(L):

@@ -442,3 +442,54 @@ def test_grouped_equals_repeated_inputs_bitwise(B, H, G, K):
         for j in range(1, H // G):
             s = s + per[:, :, j]
         assert torch.equal(g[n], s), n
+
+
+# ---------------------------------------------------------------- gate logits
+# f holds gate logits a_t and the kernels take f_t = 1 / (1 + exp(-a_t)); the
+# backward's df is dL/da_t.  The oracle evaluates the same in fp64.
+
+@pytest.mark.parametrize("variant,K,G", [("tc", 64, 0), ("tc", 128, 0), ("fast", 64, 0), ("mma", 32, 0),
+                                         ("fp32", 64, 0), ("tc", 64, 2)])
+def test_gate_logit_forward(variant, K, G):
+    mode = "fp32" if variant == "fp32" else "bf16"
+    w = Workload("gl", B=2, H=4, T=23, K=K, V=64, mode=mode, h0_range=0.5, gate_logits=True, qk_heads=G,
+                 gate_var=4.0, seed=K + G)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], f_is_logit=True,
+                             fast_tanh=variant == "fast", mma_sync=variant == "mma")
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    yr, HTr = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], f_is_logit=True)
+    _check_fwd("logit_fwd_%s_K%d_G%d" % (variant, K, G), y, HT, yr, HTr, mode)
+
+
+@pytest.mark.parametrize("mode,K,G", [("bf16", 64, 0), ("bf16", 128, 0), ("bf16", 32, 2), ("fp32", 64, 0)])
+@pytest.mark.parametrize("T,C", [(1, 16), (37, 8)])
+def test_gate_logit_backward(mode, K, G, T, C):
+    w = Workload("glb", B=2, H=4, T=T, K=K, V=64, mode=mode, h0_range=0.5, backward=True, gate_logits=True,
+                 qk_heads=G, gate_var=4.0, seed=2 * K + T + G)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    a = api()
+    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True,
+                         f_is_logit=True)
+    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=C, f_is_logit=True)
+    torch.cuda.synchronize()
+    assert a.device_status() == 0
+    gr = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], f_is_logit=True)
+    _check_grads("logit_bwd_%s_K%d_G%d_T%d" % (mode, K, G, T), g, gr, GRAD_REL if mode == "bf16" else 1e-4)
+
+
+def test_gate_logit_decode_steps_match_scan_bitwise():
+    w = Workload("gld", B=2, H=2, T=9, K=64, V=64, h0_range=0.5, gate_logits=True, seed=4)
+    xc = _cuda(make_inputs(w))
+    a = api()
+    y, HT, _ = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], f_is_logit=True)
+    H = xc["H0"].clone()
+    ys = []
+    for t in range(w.T):
+        col = lambda n: xc[n][:, :, t].contiguous()  # noqa: E731
+        ys.append(a.step(col("k"), col("v"), col("q"), col("f"), xc["W"], H, f_is_logit=True).clone())
+    torch.cuda.synchronize()
+    assert torch.equal(torch.stack(ys, 2), y) and torch.equal(H, HT)
