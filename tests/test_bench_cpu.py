@@ -1,0 +1,72 @@
+"""Host logic of bench.py (no GPU): algorithmic unit counts, the build
+fingerprint that ties a profiles/ summary to the kernel source it was taken
+from, and the parsing of the clock samples."""
+import os
+
+import pytest
+
+import bench
+from non_linear_matrix_persistent_b200 import WORKLOADS
+
+
+def test_per_step_counts_training_workload():
+    fwd, bwd = bench.per_step_counts(WORKLOADS["layer410m_train"])
+    K = V = 64
+    assert fwd["flop"] == 2 * K * V * V and bwd["flop"] == 3 * 2 * K * V * V
+    assert fwd["tanh"] == bwd["tanh"] == K * V
+    # forward: k, q, v bf16 in, f in, y fp32 out, the fp32 checkpoint every 16 steps
+    assert fwd["bytes"] == (2 * K + V) * 2 + 4 + 4 * V + 4 * K * V / 16 == 1668
+    # backward: k, q, v, dy bf16 and f in, dk, dq, dv, df fp32 out, one checkpoint read per 16 steps
+    assert bwd["bytes"] == (2 * K + 2 * V) * 2 + 4 + (2 * K + V) * 4 + 4 + 4 * K * V / 16 == 2312
+    f_only, _ = bench.per_step_counts(WORKLOADS["layer410m_fwd"])
+    assert f_only["bytes"] == 1668 - 4 * K * V / 16   # no checkpoints without a backward
+
+
+def test_kernel_digest_ignores_comments_only():
+    src = b"__global__ void k(float* p) {\n  p[0] = 1.f;  // one\n}\n"
+    same = b"/* header */\n__global__ void k(float* p)\n{\n\n  p[0] = 1.f;\n}\n// end\n"
+    other = b"__global__ void k(float* p) {\n  p[0] = 2.f;  // one\n}\n"
+    assert bench.kernel_digest(src) == bench.kernel_digest(same)
+    assert bench.kernel_digest(src) != bench.kernel_digest(other)
+
+
+def test_measured_traffic_only_for_the_profiled_build(tmp_path, monkeypatch):
+    csrc, prof = tmp_path / "csrc", tmp_path / "profiles"
+    csrc.mkdir()
+    prof.mkdir()
+    src = b"__global__ void k() {}\n"
+    (csrc / "k.cu").write_bytes(src)
+    text = "build fingerprint of k.cu: `%s` (...)\n\nDRAM traffic per launch: 1234 bytes (...)\n"
+    monkeypatch.setattr(bench, "CSRC", str(csrc))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (prof / "k.md").write_text(text % bench.kernel_digest(src))
+    assert bench.measured_traffic("k.cu", "k.md") == 1234.0
+    (prof / "k.md").write_text(text % ("0" * 16))
+    assert bench.measured_traffic("k.cu", "k.md") is None
+    assert bench.measured_traffic("k.cu", "missing.md") is None
+
+
+def test_clock_summary_parses_samples_and_reasons(tmp_path):
+    rows = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 999.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 820.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join(rows) + "\n")
+    s = bench.ClockSampler(0)
+    s.proc, s.path = object(), str(path)   # as if nvidia-smi had written the file
+    out = s.summary()
+    assert out["sm_mhz"] == 1950.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"] and out["samples"] == 3
+    assert not os.path.exists(path)
+    assert bench.ClockSampler(0).summary()["reasons"] == ["unsampled"]
+
+
+@pytest.mark.parametrize("world", [1, 4])
+def test_bench_config_names_the_workload(world):
+    w = WORKLOADS["layer410m_train"]
+    c = bench.bench_config(w, world)
+    assert c["workload"] == "layer410m_train" and c["global_batch"] == 8 * world
+    assert c["parallelism"] == "dp%d" % world and "l2" in c
