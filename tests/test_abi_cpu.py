@@ -150,6 +150,22 @@ def test_status_query_rejects_null(L):
     assert L.m2rnn_get_device_status(None, None) == _lib.ERR_INVALID_ARG
 
 
+def test_dims_struct_matches_header():
+    """The ctypes m2rnn_dims has the header's int fields in the header's order
+    (a missing or reordered field would shift every later one)."""
+    header = open(os.path.join(ROOT, "include", "m2rnn.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    body = re.search(r"typedef struct \{(.*?)\} m2rnn_dims;", header, flags=re.S).group(1)
+    names = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            assert decl.startswith("int "), decl
+            names += [n.strip() for n in decl[4:].split(",")]
+    assert names == [n for n, _ in _lib.Dims._fields_]
+    assert all(t is ctypes.c_int for _, t in _lib.Dims._fields_)
+
+
 def test_binding_signatures_match_header(L):
     """Each ctypes declaration has exactly the parameter count of the header prototype
     (a missing parameter shifts every later argument, e.g. the stream handle)."""
