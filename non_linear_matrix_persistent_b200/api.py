@@ -69,12 +69,21 @@ def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16, f_is_logit:
     return Dims(B, H, T, K, v.shape[-1], _mode(k), ckpt_stride, G if G != H else 0, int(bool(f_is_logit)))
 
 
+def _ws_key(device) -> Tuple[int, int]:
+    """Workspaces are cached per (device, stream): calls that the library
+    orders on one stream may share one, calls on different streams may
+    overlap on the GPU and must not."""
+    index = device.index if device.index is not None else torch.cuda.current_device()
+    return index, _stream(torch.device("cuda", index))
+
+
 def workspace(d: Dims, backward: bool, device) -> torch.Tensor:
-    """Zero-initialised device workspace (cached per device, grown on demand)."""
+    """Zero-initialised device workspace (cached per device and current
+    stream, grown on demand)."""
     need = _lib.lib().m2rnn_workspace_size(d, 1 if backward else 0)
     if need == 0:
         raise M2RNNError(_lib.ERR_INVALID_ARG, "m2rnn_workspace_size")
-    key = (device.index if device.index is not None else torch.cuda.current_device(), 0)
+    key = _ws_key(device)
     ws = _workspaces.get(key)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(need, dtype=torch.uint8, device=device)
@@ -181,9 +190,10 @@ def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: O
 
 
 def device_status(device=None) -> int:
-    """Synchronises the current stream and returns (and clears) the device status of the cached workspace."""
+    """Synchronises the current stream and returns (and clears) the device
+    status of the workspace cached for that stream."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
-    key = (dev.index if dev.index is not None else torch.cuda.current_device(), 0)
+    key = _ws_key(dev)
     ws = _workspaces.get(key)
     if ws is None:
         return _lib.OK

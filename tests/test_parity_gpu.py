@@ -493,3 +493,35 @@ def test_gate_logit_decode_steps_match_scan_bitwise():
         ys.append(a.step(col("k"), col("v"), col("q"), col("f"), xc["W"], H, f_is_logit=True).clone())
     torch.cuda.synchronize()
     assert torch.equal(torch.stack(ys, 2), y) and torch.equal(H, HT)
+
+
+def test_calls_on_two_streams_use_separate_workspaces():
+    """Forward + backward issued on two streams at once (each with its own
+    cached workspace) give the results of the same calls made one after the
+    other on the current stream."""
+    a = api()
+    ws = [Workload("s%d" % i, B=8, H=16, T=45, K=64, V=64, h0_range=0.5, backward=True, seed=20 + i) for i in (0, 1)]
+    xs = [_cuda(make_inputs(w)) for w in ws]
+
+    def run(x):
+        y, HT, ck = a.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=8, want_ckpt=True)
+        g = a.backward(x["k"], x["v"], x["q"], x["f"], x["W"], ck, x["dY"], ckpt_stride=8)
+        return [y, HT] + [g[n] for n in ("dk", "dv", "dq", "df", "dW", "dH0")]
+
+    ref = [run(x) for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in xs]
+    outs = []
+    for s, x in zip(streams, xs):
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            outs.append(run(x))
+    torch.cuda.synchronize()
+    for s in streams:
+        with torch.cuda.stream(s):
+            assert a.device_status() == 0
+    keys = {k for k in a._workspaces if k[1] in {s.cuda_stream for s in streams}}
+    assert len(keys) == 2
+    for o, r in zip(outs, ref):
+        for got, want in zip(o, r):
+            assert torch.equal(got, want)
