@@ -194,3 +194,19 @@ def test_api_mode_flags_are_checked_before_any_launch():
         api.forward(bf[0], bf[1], bf[2], f, W.to(torch.bfloat16), fast_tanh=True, mma_sync=True)
     with pytest.raises(ValueError):         # step needs the state buffer
         api.step(k[:, :, 0], v[:, :, 0], q[:, :, 0], f[:, :, 0], W, None)
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/m2rnn.h compiles as strict C99 (a C caller needs no C++ or CUDA headers)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "m2rnn.h"\n'
+                   "size_t ws(void) { m2rnn_dims d = {1, 1, 1, 16, 16, M2RNN_MODE_FP32_DEBUG, 16, 0, 0};\n"
+                   "  return m2rnn_workspace_size(&d, 0); }\n")
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                        os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
