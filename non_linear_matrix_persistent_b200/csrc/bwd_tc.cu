@@ -42,6 +42,13 @@
 // per CTA are summed over the batch and slices in a fixed order by a
 // separate kernel, so results are deterministic.
 //
+// Input variants: with grouped k and q the producer copies the rows of the
+// pair's head group (qk_pair) and dk, dq go to per-head workspace rows that
+// m2rnn_qk_group_reduce_kernel sums per group; with gate logits the ring gets
+// f_t = 1 / (1 + exp(-a_t)) (gate_value) and the storer writes dL/da_t =
+// dL/df_t · f_t (1 - f_t) (gate_grad).  The epilogue stays scalar: packed
+// fp32 pairs, which help the forward, measured slower here.
+//
 // Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16.
 #include <cuda_bf16.h>
 

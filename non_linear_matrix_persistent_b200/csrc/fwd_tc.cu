@@ -41,6 +41,13 @@
 // producer warp (k, q, v and f for TC steps per ring stage), one MMA warp
 // (also owns the TMEM allocation) and one storer warp that sums the partial
 // readouts and writes y.
+//
+// Input variants are resolved where the producer loads a step's inputs: with
+// grouped k and q the pair reads the rows of its head group (qk_pair), and
+// with gate logits the ring receives f_t = 1 / (1 + exp(-a_t)) (gate_value),
+// so the epilogue is the same for every variant.  The epilogue's elementwise
+// arithmetic runs on packed fp32 pairs (FADD2 / FFMA2), except in the
+// fast-tanh kernel at V = 128, where the scalar loop measured faster.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
