@@ -160,11 +160,18 @@ def measured_traffic(kernel_file: str, profile_md: str):
     return None
 
 
-def _sample_pairs(w, cores, budget_flop):
+def _sample_pairs(w, cores):
+    """One distinct (b, h) pair per host thread (the oracle runs one pair per
+    thread), at most all of them: pair i of the sample is number
+    (i · s) mod B·H for a stride s coprime to B·H, spread over the batch and
+    heads."""
+    import math
     pairs_total = w.B * w.H
-    per_pair = 2.0 * w.T * w.K * w.V * w.V * (4.0 if w.backward else 1.0)
-    npairs = int(max(1, min(pairs_total, cores, budget_flop // per_pair)))
-    return [(i % w.B, (i * 7) % w.H) for i in range(npairs)]
+    npairs = max(1, min(pairs_total, cores))
+    s = 37
+    while math.gcd(s, pairs_total) != 1:
+        s += 1
+    return [divmod((i * s) % pairs_total, w.H) for i in range(npairs)]
 
 
 def _oracle_sample(w, pairs, cores):
@@ -195,8 +202,8 @@ def bench_config(w, world):
 def run_reference(args, w):
     """fp64 CPU oracle on a bounded sample of (b, h) pairs at full length."""
     from oracle import oracle
-    cores = oracle.default_threads()
-    pairs = _sample_pairs(w, cores, float(os.environ.get("M2RNN_REF_FLOP_BUDGET", 2.0e10)))
+    pairs = _sample_pairs(w, oracle.default_threads())
+    cores = len(pairs)   # threads that run
     run = _oracle_sample(w, pairs, cores)
     times = []
     for it in range(args.warmup + args.steps):
@@ -218,8 +225,8 @@ def run_reference(args, w):
 
 def cpu_baseline(w):
     from oracle import oracle
-    cores = oracle.default_threads()
-    pairs = _sample_pairs(w, cores, 2.0e10)
+    pairs = _sample_pairs(w, oracle.default_threads())
+    cores = len(pairs)   # threads that run
     run = _oracle_sample(w, pairs, cores)
     t0 = time.perf_counter()
     run()

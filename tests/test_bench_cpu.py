@@ -70,3 +70,13 @@ def test_bench_config_names_the_workload(world):
     c = bench.bench_config(w, world)
     assert c["workload"] == "layer410m_train" and c["global_batch"] == 8 * world
     assert c["parallelism"] == "dp%d" % world and "l2" in c
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+@pytest.mark.parametrize("cores", [1, 3, 16, 500])
+def test_cpu_sample_is_one_distinct_pair_per_thread(name, cores):
+    w = WORKLOADS[name]
+    pairs = bench._sample_pairs(w, cores)
+    assert len(pairs) == min(cores, w.B * w.H)
+    assert len(set(pairs)) == len(pairs)
+    assert all(0 <= b < w.B and 0 <= h < w.H for b, h in pairs)
