@@ -210,3 +210,25 @@ def test_header_is_plain_c(tmp_path):
                         os.path.join(ROOT, "include"), "-c", str(src), "-o", str(tmp_path / "use.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_api_rejects_bad_tensors_before_any_launch():
+    """Shape, dtype and device problems are reported by the binding before it
+    allocates a workspace or calls the library (CPU tensors stand in for any
+    tensor that is not on the expected CUDA device)."""
+    import torch
+    from non_linear_matrix_persistent_b200 import api
+    B, H, T, K, V = 1, 2, 3, 16, 16
+    bf = dict(dtype=torch.bfloat16)
+    k, q = torch.zeros(B, H, T, K, **bf), torch.zeros(B, H, T, K, **bf)
+    v, W = torch.zeros(B, H, T, V, **bf), torch.zeros(H, V, V, **bf)
+    f = torch.zeros(B, H, T)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.forward(k, v, q, f, W)
+    with pytest.raises(TypeError):                  # integer inputs select no mode
+        api.forward(k.to(torch.int32), v, q, f, W)
+    with pytest.raises(ValueError):                 # k with a head count that does not divide H
+        api.dims_of(torch.zeros(B, 3, T, K, **bf), v)
+    d = api.dims_of(k, v, ckpt_stride=4, f_is_logit=True)
+    assert (d.B, d.H, d.T, d.K, d.V, d.ckpt_stride, d.qk_heads, d.f_is_logit) == (B, H, T, K, V, 4, 0, 1)
+    assert d.mode == 0 and api.dims_of(k.float(), v.float()).mode == 1
