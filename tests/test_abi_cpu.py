@@ -232,3 +232,18 @@ def test_api_rejects_bad_tensors_before_any_launch():
     d = api.dims_of(k, v, ckpt_stride=4, f_is_logit=True)
     assert (d.B, d.H, d.T, d.K, d.V, d.ckpt_stride, d.qk_heads, d.f_is_logit) == (B, H, T, K, V, 4, 0, 1)
     assert d.mode == 0 and api.dims_of(k.float(), v.float()).mode == 1
+
+
+def test_enum_values_match_header():
+    """Status codes and modes of the binding carry the header's values."""
+    header = open(os.path.join(ROOT, "include", "m2rnn.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    vals = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(M2RNN_[A-Z0-9_]+)\s*=\s*(\d+)", header)}
+    py = {"M2RNN_OK": _lib.OK, "M2RNN_ERR_INVALID_ARG": _lib.ERR_INVALID_ARG,
+          "M2RNN_ERR_UNSUPPORTED_SHAPE": _lib.ERR_UNSUPPORTED_SHAPE, "M2RNN_ERR_MISALIGNED": _lib.ERR_MISALIGNED,
+          "M2RNN_ERR_WORKSPACE": _lib.ERR_WORKSPACE, "M2RNN_ERR_CUDA": _lib.ERR_CUDA,
+          "M2RNN_ERR_DEVICE_TIMEOUT": _lib.ERR_DEVICE_TIMEOUT,
+          "M2RNN_MODE_BF16_TC": _lib.MODE_BF16_TC, "M2RNN_MODE_FP32_DEBUG": _lib.MODE_FP32_DEBUG,
+          "M2RNN_MODE_BF16_TC_FAST_TANH": _lib.MODE_BF16_TC_FAST_TANH,
+          "M2RNN_MODE_BF16_MMA_SYNC": _lib.MODE_BF16_MMA_SYNC}
+    assert vals == py
