@@ -80,3 +80,14 @@ def test_cpu_sample_is_one_distinct_pair_per_thread(name, cores):
     assert len(pairs) == min(cores, w.B * w.H)
     assert len(set(pairs)) == len(pairs)
     assert all(0 <= b < w.B and 0 <= h < w.H for b, h in pairs)
+
+
+def test_launches_per_step():
+    from non_linear_matrix_persistent_b200 import build
+    build.build()   # the workspace query needs the library (it launches nothing)
+    # training: forward, backward, dW reduction; 128 pairs fill the GPU, so rows are not split
+    assert bench.launches_per_step(WORKLOADS["layer410m_train"]) == 3
+    assert bench.launches_per_step(WORKLOADS["layer410m_fwd"]) == 1
+    # 16 pairs: the forward splits rows and sums the slices' readouts in a second kernel
+    assert bench.launches_per_step(WORKLOADS["long_b1_fwd"]) == 2
+    assert bench.launches_per_step(WORKLOADS["tiny_fp32"]) == 1
