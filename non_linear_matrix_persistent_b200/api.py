@@ -19,7 +19,6 @@ contiguous CUDA tensors with the head-first layouts of the header.
 """
 from __future__ import annotations
 
-import math
 from typing import Dict, Optional, Tuple
 
 import torch

@@ -9,7 +9,6 @@ No GPU fault, trap or hang is involved.
 """
 import numpy as np
 import pytest
-import torch
 
 from non_linear_matrix_persistent_b200 import Workload, make_inputs
 from oracle import oracle

@@ -10,7 +10,6 @@ dropped, the readout taken before the update, and in the backward a dropped
 f_t in the carry of G, a missing tanh derivative, the sign of df, dq from the
 previous state and a transposed W in the carry.
 """
-import os
 import subprocess
 
 import pytest

@@ -8,8 +8,6 @@ m2rnn_backward's on the same inputs, call after call (the array keeps the
 previous call's contents).  This file is collected last so that a failure
 here leaves every other test already run.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
