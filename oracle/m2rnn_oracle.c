@@ -17,7 +17,7 @@
  * same pair with garbled LaTeX).  H_t is K×V (same §2.1: matrix-valued
  * state), W is V×V per head (it right-multiplies H_{t-1}; §2.2 gives the GEMM
  * dimensions (K, V, V)), f_t is a scalar in [0,1] that depends only on the
- * input (§2.1 forget gate).  The pages define no readout: (3) is this build's
+ * input (§2.1 forget gate).  The pages define no readout: (3) is the library's
  * stated reading, using the updated state H_t.
  *
  * Indexing: array step t (0-based) consumes k[t], v[t], q[t], f[t] and

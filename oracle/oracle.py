@@ -8,7 +8,7 @@ with it.
 The recurrence it evaluates is the one of "M²RNN: Non-Linear RNNs with
 Matrix-Valued States for Scalable Language Modeling" (gist.science technical
 summary §2.1: Z_t = tanh(H_{t-1}W + k_t v_tᵀ), H_t = f_t H_{t-1} + (1-f_t) Z_t),
-plus the readout y_t = H_tᵀ q_t, a reading of this build because the pages
+plus the readout y_t = H_tᵀ q_t, the library's reading because the pages
 define no readout.  The backward is the exact chain rule of the same three
 equations.  Every function here is pinned by tests/test_oracle_pins.py
 against closed forms, invariants, torch.nn.RNN (f = 0) and finite
