@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 from non_linear_matrix_persistent_b200 import WORKLOADS, make_inputs  # noqa: E402
 from non_linear_matrix_persistent_b200.inputs import make_shard_inputs  # noqa: E402
 
-METRIC = "M2RNN layer fwd(+bwd) tokens/s on 1 B200"
+METRIC = "M2RNN layer fwd(+bwd) tokens/s on 1 B200; tensor-pipe % and HBM GB/s via ncu"
 DEFAULT_WORKLOAD = "layer410m_train"
 CKPT_STRIDE = 16
 L2_FLUSH_BYTES = 256 << 20
