@@ -42,8 +42,15 @@ DEFAULT_WORKLOAD = "layer410m_train"
 CKPT_STRIDE = 16
 L2_FLUSH_BYTES = 256 << 20
 NUM_SMS = 148
-SFU_PER_SM_PER_CLK = 16      # special-function (exp / reciprocal) results per SM per clock
-SFU_PER_TANH = 2             # tanh = 1 - 2/(1 + e^{2x}): one exp and one reciprocal
+SFU_PER_SM_PER_CLK = 16      # special-function (exp / reciprocal / tanh) results per SM per clock
+# SFU operations the kernels spend per tanh: the accurate tanh is 1 - 2/(1 + e^{2x})
+# (one exp and one reciprocal), the fast-tanh inference mode one tanh.approx.
+# This is an implementation cost; the roofline fraction counts the method's
+# work, one tanh per state element and step.
+SFU_OPS_PER_TANH = {"accurate": 2, "fast": 1}
+# Forward-only workloads timed beside the training step (each its own CUDA-event
+# timing, L2 flushed between steps).
+FORWARD_CONFIGS = ("tiny_fp32", "layer410m_fwd", "long_b1_fwd", "layer7b_moe_fwd")
 CSRC = os.path.join(ROOT, "non_linear_matrix_persistent_b200", "csrc")
 
 
@@ -156,11 +163,26 @@ def kernel_digest(src: bytes) -> str:
     return hashlib.sha256((code + "\n" + flags).encode()).hexdigest()[:16]
 
 
+# Headers every kernel file includes; a profile is tied to them as well.
+KERNEL_HEADERS = ("common.cuh", "ptx.cuh", "tc_common.cuh", "kernels.h")
+
+
+def kernel_source(kernel_file: str) -> bytes:
+    """The kernel file followed by the shared headers it is compiled with."""
+    parts = [open(os.path.join(CSRC, kernel_file), "rb").read()]
+    for h in KERNEL_HEADERS:
+        path = os.path.join(CSRC, h)
+        if os.path.exists(path):
+            parts.append(open(path, "rb").read())
+    return b"\n".join(parts)
+
+
 def measured_traffic(kernel_file: str, profile_md: str):
     """DRAM bytes per launch recorded in a profiles/ summary, when that summary
-    was taken from the current kernel build (kernel_digest); else None."""
+    was taken from the current kernel build (kernel_digest of the kernel file
+    and its headers); else None."""
     try:
-        src = open(os.path.join(CSRC, kernel_file), "rb").read()
+        src = kernel_source(kernel_file)
         text = open(os.path.join(ROOT, "profiles", profile_md)).read()
     except OSError:
         return None
@@ -202,6 +224,79 @@ def _oracle_sample(w, pairs, cores):
         else:
             oracle.forward(*args, nthreads=cores)
     return run
+
+
+def kernel_entry(ms_mean, cnt, units, T, peaks, peak_kind, sm_max, sm_mhz, tanh_kind="accurate", traffic=None):
+    """Roofline figures of one kernel from its mean CUDA-event time.
+
+    The bound is the special-function unit: the method evaluates one tanh per
+    state element and step (K·V per (b, h, t)), and the derived peak is
+    148 SMs x 16 results per SM per clock x the maximum SM clock.  The SFU
+    operations the implementation spends per tanh are reported apart
+    (`sfu_ops`); the tensor-pipe and HBM fractions of the same launch go beside
+    them.  `units` is the (b, h, t) steps one launch processes."""
+    s = ms_mean / 1e3
+    tanh_rate = cnt["tanh"] * units / s / 1e9
+    sfu_peak = NUM_SMS * SFU_PER_SM_PER_CLK * sm_max * 1e6 / 1e9
+    per = SFU_OPS_PER_TANH[tanh_kind]
+    e = {
+        "ms": ms_mean,
+        "bound": "alu", "unit": "Gtanh/s", "achieved": tanh_rate, "peak": sfu_peak, "frac": tanh_rate / sfu_peak,
+        "peak_source": "derived: %d SMs x %d SFU results/clk x %.0f MHz (one tanh per state element and step)" % (
+            NUM_SMS, SFU_PER_SM_PER_CLK, sm_max),
+        "sfu_ops": {"per_tanh": per, "achieved_gops": per * tanh_rate, "frac": per * tanh_rate / sfu_peak},
+        "traffic": traffic,
+        "algorithmic_per_step": cnt,
+        "units_per_launch": units,
+        "hbm": {"achieved_gbs": cnt["bytes"] * units / s / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                "frac": cnt["bytes"] * units / s / 1e9 / peaks["hbm_gbs"], "peak_kind": peak_kind},
+        "cycles_per_recurrence_step": s * sm_mhz * 1e6 / T,
+    }
+    if cnt.get("flop"):
+        tf = cnt["flop"] * units / s / 1e12
+        e["tensor"] = {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
+                       "frac": tf / peaks["bf16_tflops"], "peak_kind": peak_kind}
+    return e
+
+
+def time_forward_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_max, sm_mhz):
+    """One forward-only workload: the default forward (and, for bf16 inputs,
+    the fast-tanh inference forward) timed per step with CUDA events on the
+    launching stream, L2 flushed between steps."""
+    from non_linear_matrix_persistent_b200 import api
+    w = WORKLOADS[name]
+    x = make_inputs(w, device=str(dev))
+    B, H, T, K, V = w.B, w.H, w.T, w.K, w.V
+    out = {"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev)}
+    stream = torch.cuda.current_stream(dev)
+    variants = [("accurate", False)] + ([("fast", True)] if w.mode == "bf16" else [])
+    res = {"B": B, "H": H, "T": T, "K": K, "V": V, "mode": w.mode, "tokens": B * T}
+    for kind, fast in variants:
+        def run():
+            api.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], out=out, fast_tanh=fast)
+        for _ in range(warmup):
+            run()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            run()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if api.device_status(dev) != 0:
+            raise RuntimeError("device-side wait ran out in the %s forward" % name)
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        cnt, _ = per_step_counts(w)
+        if w.mode != "bf16":
+            cnt = dict(cnt, flop=0.0)   # the fp32 debug mode runs on CUDA cores
+        traffic = measured_traffic("fwd_tc.cu", "m2rnn_fwd_tc_%s.md" % name) if kind == "accurate" else None
+        e = kernel_entry(ms, cnt, B * H * T, T, peaks, peak_kind, sm_max, sm_mhz, kind, traffic)
+        e["tokens_per_s"] = B * T / (ms / 1e3)
+        e["steps"] = steps
+        res["forward" if kind == "accurate" else "forward_fast_tanh"] = e
+    del x, out
+    return res
 
 
 def bench_config(w, world):
@@ -257,6 +352,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the main workload (no forward-only configs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -402,30 +499,24 @@ def main():
     units = B * H * T   # (b, h, t) steps per launch on this rank
     kernels = {}
     for name, ms_list, cnt, src, prof in (
-            ("m2rnn_fwd_tc_kernel", fwd_ms, cf, "fwd_tc.cu", "m2rnn_fwd_tc_layer410m_train.md"),
-            ("m2rnn_bwd_tc_kernel", bwd_ms, cb, "bwd_tc.cu", "m2rnn_bwd_tc_layer410m_train.md")):
+            ("m2rnn_fwd_tc_kernel", fwd_ms, cf, "fwd_tc.cu", "m2rnn_fwd_tc_%s.md" % w.name),
+            ("m2rnn_bwd_tc_kernel", bwd_ms, cb, "bwd_tc.cu", "m2rnn_bwd_tc_%s.md" % w.name)):
         if name.startswith("m2rnn_bwd") and not w.backward:
             continue
-        s = statistics.mean(ms_list) / 1e3
-        sfu = SFU_PER_TANH * cnt["tanh"] * units / s / 1e9
-        sfu_peak = NUM_SMS * SFU_PER_SM_PER_CLK * sm_max * 1e6 / 1e9
-        traffic = measured_traffic(src, prof) if w.name == "layer410m_train" else None
-        kernels[name] = {
-            "ms": s * 1e3,
-            "bound": "alu", "unit": "GSFUop/s", "achieved": sfu, "peak": sfu_peak, "frac": sfu / sfu_peak,
-            "peak_source": "derived: %d SMs x %d SFU results/clk x %.0f MHz; %d SFU ops per tanh" % (
-                NUM_SMS, SFU_PER_SM_PER_CLK, sm_max, SFU_PER_TANH),
-            "traffic": traffic,
-            "algorithmic_per_step": cnt,
-            "tensor": {"achieved_tflops": cnt["flop"] * units / s / 1e12, "peak_tflops": peaks["bf16_tflops"],
-                       "frac": cnt["flop"] * units / s / 1e12 / peaks["bf16_tflops"], "peak_kind": peak_kind},
-            "hbm": {"achieved_gbs": cnt["bytes"] * units / s / 1e9, "peak_gbs": peaks["hbm_gbs"],
-                    "frac": cnt["bytes"] * units / s / 1e9 / peaks["hbm_gbs"], "peak_kind": peak_kind},
-            "cycles_per_recurrence_step": s * sm_mhz * 1e6 / T,
-        }
+        kernels[name] = kernel_entry(statistics.mean(ms_list), cnt, units, T, peaks, peak_kind, sm_max, sm_mhz,
+                                     "accurate", measured_traffic(src, prof))
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     roofline = dict(kernel=dom, **{k: v for k, v in kernels[dom].items()})
     roofline["kernels"] = kernels
+
+    # Forward-only workloads on the same clock (rank 0 of a single-GPU run).
+    forward_configs = None
+    if world == 1 and not args.no_extra:
+        fsteps = max(3, min(args.steps, 10))
+        forward_configs = {}
+        for name in FORWARD_CONFIGS:
+            forward_configs[name] = time_forward_config(name, fsteps, args.warmup, dev, flush, peaks, peak_kind,
+                                                        sm_max, sm_mhz)
     launches = args.steps * launches_per_step(w)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -437,6 +528,8 @@ def main():
                     "how": "pinned host inputs -> device -> fwd+bwd -> all results to pinned host, every step; "
                            "3 streams, 2 buffer sets (step i compute overlaps i+1 copy-in and i-1 copy-out)"},
             "roofline": roofline}
+    if forward_configs is not None:
+        line["forward_configs"] = forward_configs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -126,7 +126,9 @@ size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward);
  * H0 and HT may be the same buffer: every element of H0 is read before the
  * same element of HT is written, so the state can be advanced in place --
  * with T = 1 this is one decode step, and T such calls give the scan's y and
- * H_T bit for bit. */
+ * H_T bit for bit.  This is the library's single-step decode: there is no
+ * separate step entry point (the Python binding's step() is this call with
+ * T = 1 and H0 == HT). */
 m2rnn_status m2rnn_forward(const m2rnn_dims* d,
                            const void* k, const void* v, const void* q,
                            const float* f, const void* W, const float* H0,
@@ -137,7 +139,10 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d,
  * (NULL = 0; dHT and dH0 may be the same buffer).  ckpt must come from
  * m2rnn_forward with the same inputs and
  * the same dims (including ckpt_stride); the states inside each chunk of C
- * steps are recomputed from it.  Writes dk, dv, dq, df, dW, dH0 (all
+ * steps are recomputed from it.  The initial state H_0 is not an argument:
+ * it is ckpt[b][h][0], which m2rnn_forward writes from its H0 (zeros for a
+ * NULL H0), so the recomputation always starts from the state the forward
+ * used and a second copy of H_0 cannot disagree with the checkpoints.  Writes dk, dv, dq, df, dW, dH0 (all
  * required, all fp32).  M2RNN_MODE_BF16_TC supports V = 64, K in
  * {32, 64, 128} and ckpt_stride <= 16 (other shapes return
  * M2RNN_ERR_UNSUPPORTED_SHAPE); M2RNN_MODE_FP32_DEBUG supports every shape. */
@@ -151,17 +156,21 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d,
 
 /* Allocation-free m2rnn_backward (the pages describe no such variant: it is
  * an interface addition of this library).  For callers that cannot allocate
- * device memory when they need gradients, e.g. code running under CUDA-graph
- * capture or services that forbid allocator calls after start-up.  Same
- * arguments and results as m2rnn_backward minus the workspace: the scratch
- * comes from a 32 MiB array compiled into the library, which every GPU that
- * loads the library keeps until the process exits.
+ * device memory when they need gradients: services that forbid allocator
+ * calls after start-up (an allocation can synchronise the device or fail
+ * under memory pressure) and hosts that hand the library only the tensors
+ * they already own.  Same arguments and results (bit for bit) as
+ * m2rnn_backward minus the workspace: the scratch comes from a 32 MiB array
+ * compiled into the library, which every GPU that loads the library keeps
+ * until the process exits.
  *  - Problems with m2rnn_workspace_size(d, 1) > 32 MiB return
  *    M2RNN_ERR_WORKSPACE and launch nothing.
  *  - All calls share the array: calls whose kernels overlap on the GPU race
  *    and give wrong results; order them on one stream.
  *  - The first call on a device looks up the array's device address (no
- *    allocation); make it before any stream capture starts.
+ *    allocation); make it before any stream capture starts.  The address is
+ *    cached per device for the life of the process: do not use this entry
+ *    point across a device reset.
  *  - Device-side wait timeouts are not reported by this entry point. */
 m2rnn_status m2rnn_backward_noalloc(const m2rnn_dims* d,
                                     const void* k, const void* v, const void* q,

@@ -1,10 +1,10 @@
 // Allocation-free variant of m2rnn_backward.
 //
 // Some callers cannot allocate device memory at the point where they need
-// gradients: code running while a CUDA graph is being captured, real-time or
-// embedded services that forbid allocator calls after start-up (an allocation
-// can synchronise the device or fail under memory pressure), or hosts that
-// hand this library only the tensors they already own.  m2rnn_backward needs
+// gradients: real-time or embedded services that forbid allocator calls after
+// start-up (an allocation can synchronise the device or fail under memory
+// pressure), or hosts that hand this library only the tensors they already
+// own.  m2rnn_backward needs
 // a caller-allocated workspace for its scratch (the device status word, the
 // per-(b, h) dW partials and the per-CTA recompute buffer); this entry point
 // takes that scratch from a fixed array compiled into the library instead, so
@@ -21,7 +21,8 @@
 //    their streams) race on it and produce garbage;
 //  * the first call on a device looks up the array's device address (a CUDA
 //    runtime query, no allocation); make that first call before any stream
-//    capture begins;
+//    capture begins.  The address is cached per device for the life of the
+//    process, so the entry point must not be used across a device reset;
 //  * a device-side wait that runs out is recorded in the array's status word,
 //    which this entry point clears at the start of each call and does not
 //    report (m2rnn_backward with your own workspace does).

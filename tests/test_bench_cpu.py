@@ -91,3 +91,37 @@ def test_launches_per_step():
     # 16 pairs: the forward splits rows and sums the slices' readouts in a second kernel
     assert bench.launches_per_step(WORKLOADS["long_b1_fwd"]) == 2
     assert bench.launches_per_step(WORKLOADS["tiny_fp32"]) == 1
+
+
+def test_roofline_fraction_counts_one_tanh_per_element():
+    """frac is the method's tanh rate (K·V per (b, h, t)) over the derived SFU
+    peak; the implementation's SFU operations per tanh are reported apart."""
+    w = WORKLOADS["layer410m_train"]
+    fwd, _ = bench.per_step_counts(w)
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}
+    units = w.B * w.H * w.T
+    ms = 2.0
+    e = bench.kernel_entry(ms, fwd, units, w.T, peaks, "measured", 1965.0, 1965.0, "accurate")
+    tanh_rate = 64 * 64 * units / (ms / 1e3) / 1e9
+    peak = 148 * 16 * 1965.0 / 1e3
+    assert e["unit"] == "Gtanh/s" and abs(e["achieved"] - tanh_rate) < 1e-9 * tanh_rate
+    assert abs(e["peak"] - peak) < 1e-9 and abs(e["frac"] - tanh_rate / peak) < 1e-12
+    assert e["sfu_ops"]["per_tanh"] == 2 and abs(e["sfu_ops"]["frac"] - 2 * e["frac"]) < 1e-12
+    fast = bench.kernel_entry(ms, fwd, units, w.T, peaks, "measured", 1965.0, 1965.0, "fast")
+    assert fast["frac"] == e["frac"] and fast["sfu_ops"]["per_tanh"] == 1
+    assert abs(e["tensor"]["achieved_tflops"] - 2 * 64 ** 3 * units / 2e-3 / 1e12) < 1e-6
+    assert abs(e["cycles_per_recurrence_step"] - 2e-3 * 1965e6 / w.T) < 1e-6
+    # a CUDA-core (fp32 debug) kernel has no tensor-pipe figure
+    assert "tensor" not in bench.kernel_entry(ms, dict(fwd, flop=0.0), units, w.T, peaks, "measured",
+                                              1965.0, 1965.0)
+
+
+def test_kernel_digest_covers_the_shared_headers(tmp_path, monkeypatch):
+    csrc = tmp_path / "csrc"
+    csrc.mkdir()
+    (csrc / "k.cu").write_bytes(b"__global__ void k() {}\n")
+    (csrc / "ptx.cuh").write_bytes(b"#define A 1\n")
+    monkeypatch.setattr(bench, "CSRC", str(csrc))
+    d1 = bench.kernel_digest(bench.kernel_source("k.cu"))
+    (csrc / "ptx.cuh").write_bytes(b"#define A 2\n")
+    assert bench.kernel_digest(bench.kernel_source("k.cu")) != d1

@@ -1,14 +1,16 @@
 """m2rnn_backward_noalloc: the allocation-free backward entry point.
 
 For callers that cannot allocate device memory when they need gradients
-(code under CUDA-graph capture, services that forbid allocator calls after
-start-up).  The entry point takes its scratch from an array compiled into the
-library instead of a caller workspace; its gradients must match
-m2rnn_backward's on the same inputs, call after call (the array keeps the
-previous call's contents).  This file is collected last so that a failure
-here leaves every other test already run.
+(services that forbid allocator calls after start-up, because an allocation
+can synchronise the device or fail under memory pressure, and hosts that hand
+the library only the tensors they already own).  The entry point takes its
+scratch from an array compiled into the library instead of a caller
+workspace.  It runs the same deterministic kernels as m2rnn_backward (every
+reduction in a fixed order), so its gradients must equal m2rnn_backward's bit
+for bit on the same inputs, call after call (the array keeps the previous
+call's contents).  This file is collected last so that a failure here leaves
+every other test already run.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -16,7 +18,6 @@ from non_linear_matrix_persistent_b200 import Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-GRAD_REL = 1e-2
 NAMES = ("dk", "dv", "dq", "df", "dW", "dH0")
 
 
@@ -55,11 +56,9 @@ def test_noalloc_backward_matches_workspace_backward(mode):
         assert st == _lib.OK, _lib.status_string(st)
         torch.cuda.synchronize()
         for n in NAMES:
-            got = out[n].double().cpu().numpy()
-            r = ref[n].double().cpu().numpy()
-            assert np.isfinite(got).all(), (call, n)
-            rel = np.linalg.norm(got - r) / max(np.linalg.norm(r), 1e-300)
-            assert rel <= GRAD_REL, (call, n, rel)
+            assert torch.isfinite(out[n]).all(), (call, n)
+            # same kernels, same order of every sum: identical bits
+            assert torch.equal(out[n], ref[n]), (call, n, float((out[n] - ref[n]).abs().max()))
 
 
 def test_noalloc_rejects_problems_larger_than_its_array():
