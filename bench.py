@@ -51,6 +51,8 @@ SFU_OPS_PER_TANH = {"accurate": 2, "fast": 1}
 # Forward-only workloads timed beside the training step (each its own CUDA-event
 # timing, L2 flushed between steps).
 FORWARD_CONFIGS = ("tiny_fp32", "layer410m_fwd", "long_b1_fwd", "layer7b_moe_fwd")
+# Training workloads (forward with checkpoints + backward) timed beside the main one.
+TRAINING_CONFIGS = ("layer7b_moe_train",)
 CSRC = os.path.join(ROOT, "non_linear_matrix_persistent_b200", "csrc")
 
 
@@ -299,6 +301,51 @@ def time_forward_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_ma
     return res
 
 
+def time_training_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_max, sm_mhz):
+    """One training workload: the forward with checkpoints and the backward,
+    each timed per step with CUDA events on the launching stream, L2 flushed
+    between steps."""
+    from non_linear_matrix_persistent_b200 import api
+    w = WORKLOADS[name]
+    x = make_inputs(w, device=str(dev))
+    B, H, T, K, V, C = w.B, w.H, w.T, w.K, w.V, CKPT_STRIDE
+    out = {"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev),
+           "ckpt": torch.empty(B, H, (T + C - 1) // C, K, V, device=dev)}
+    gout = {}
+    stream = torch.cuda.current_stream(dev)
+
+    def run(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], ckpt_stride=C, want_ckpt=True, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+        gout.update(api.backward(x["k"], x["v"], x["q"], x["f"], x["W"], out["ckpt"], x["dY"], ckpt_stride=C,
+                                 out=gout))
+        if ev is not None:
+            ev[2].record(stream)
+    for _ in range(warmup):
+        run()
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for ev in evs:
+        flush.zero_()
+        run(ev)
+    torch.cuda.synchronize()
+    if api.device_status(dev) != 0:
+        raise RuntimeError("device-side wait ran out in the %s step" % name)
+    fwd = statistics.mean(a.elapsed_time(b) for a, b, c in evs)
+    bwd = statistics.mean(b.elapsed_time(c) for a, b, c in evs)
+    cf, cb = per_step_counts(w)
+    units = B * H * T
+    res = {"B": B, "H": H, "T": T, "K": K, "V": V, "ckpt_stride": C, "tokens": B * T, "steps": steps,
+           "ms_per_step": fwd + bwd, "tokens_per_s": B * T / ((fwd + bwd) / 1e3),
+           "forward": kernel_entry(fwd, cf, units, T, peaks, peak_kind, sm_max, sm_mhz),
+           "backward": kernel_entry(bwd, cb, units, T, peaks, peak_kind, sm_max, sm_mhz)}
+    del x, out, gout
+    return res
+
+
 def bench_config(w, world):
     """The workload description both arms print (same keys, same values)."""
     return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "K": w.K, "V": w.V, "ckpt_stride": CKPT_STRIDE,
@@ -517,6 +564,10 @@ def main():
         for name in FORWARD_CONFIGS:
             forward_configs[name] = time_forward_config(name, fsteps, args.warmup, dev, flush, peaks, peak_kind,
                                                         sm_max, sm_mhz)
+        training_configs = {}
+        for name in TRAINING_CONFIGS:
+            training_configs[name] = time_training_config(name, max(3, min(args.steps, 5)), args.warmup, dev,
+                                                          flush, peaks, peak_kind, sm_max, sm_mhz)
     launches = args.steps * launches_per_step(w)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -530,6 +581,7 @@ def main():
             "roofline": roofline}
     if forward_configs is not None:
         line["forward_configs"] = forward_configs
+        line["training_configs"] = training_configs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

@@ -49,7 +49,8 @@
 // dL/df_t · f_t (1 - f_t) (gate_grad).  The epilogue stays scalar: packed
 // fp32 pairs, which help the forward, measured slower here.
 //
-// Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16.
+// Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16; the other
+// shapes run the general-shape kernel of bwd_tcg.cu.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -755,22 +756,32 @@ static cudaError_t launch_bwd_tc_k(const Params& p0, cudaStream_t stream) {
     return launch_dw_reduce(p, stream);
 }
 
-int bwd_tc_slices(int K) { return K > 64 ? 2 : 1; }
-
-bool bwd_tc_supported(int K, int V, int C) {
+namespace {
+// Shapes of this file's kernel (the extended operands need V = 64 and tiles
+// of at least 16 rows); every other shape goes to the general-shape kernel of
+// bwd_tcg.cu.
+bool bwd_tcx_supported(int K, int V, int C) {
     return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64, 1>::CMAX;
 }
+}  // namespace
+
+int bwd_tc_slices(int K, int V) {
+    if (bwd_tcx_supported(K, V, 1)) return K > 64 ? 2 : 1;
+    return bwd_tcg_slices(K, V);
+}
+
+bool bwd_tc_supported(int K, int V, int C) { return bwd_tcx_supported(K, V, C) || bwd_tcg_supported(K, V, C); }
 
 // Per (b, h): dW partials of each slice, and the recompute scratch of
 // 2·C·K·V values (C states and C Z's of a chunk).
-size_t bwd_tc_workspace(int B, int H, int K, int V, int C) {
-    if (!bwd_tc_supported(K, V, C)) return 0;
-    const size_t nsl = (size_t)bwd_tc_slices(K);
+size_t bwd_tc_workspace(int B, int H, int T, int K, int V, int C) {
+    if (!bwd_tcx_supported(K, V, C)) return bwd_tcg_workspace(B, H, T, K, V, C);
+    const size_t nsl = (size_t)bwd_tc_slices(K, V);
     return sizeof(float) * ((size_t)B * H * nsl * V * V + (size_t)B * H * 2 * C * K * V);
 }
 
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s) {
-    if (!bwd_tc_supported(p.K, p.V, p.C)) return cudaErrorNotSupported;
+    if (!bwd_tcx_supported(p.K, p.V, p.C)) return launch_bwd_tcg(p, s);
     switch (p.K) {
         case 32: return launch_bwd_tc_k<32, 1>(p, s);
         case 64: return launch_bwd_tc_k<64, 1>(p, s);

@@ -42,6 +42,8 @@ struct Params {
     int fast_tanh;      // forward: tanh.approx.f32 instead of the exp-based tanh
     float* ypart;       // forward with slices > 1: [slices][B*H][T][V] partial readouts (workspace)
     float* scratch;     // per-CTA recompute scratch (workspace)
+    float* dv_part;     // backward with slices > 1 (general-shape kernel): [slices][B*H][T][V] (workspace)
+    float* df_part;     // same: [slices][B*H][T] (workspace)
     uint32_t* status;   // device status word (workspace)
     uint64_t wait_limit_ns;
     int fault;          // injected fault (m2rnn_debug_set_fault), 0 = none

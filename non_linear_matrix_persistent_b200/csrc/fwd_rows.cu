@@ -1,0 +1,277 @@
+// M²RNN forward scan for few (b, h) pairs: one warp per state row, CUDA-core
+// FFMA, no per-step barrier.
+//
+// Recurrence (gist.science technical summary of "M²RNN: Non-Linear RNNs with
+// Matrix-Valued States for Scalable Language Modeling", §2.1):
+//   Z_t = tanh(H_{t-1} W + k_t v_tᵀ),  H_t = f_t H_{t-1} + (1 - f_t) Z_t,
+// plus the readout y_t = H_tᵀ q_t (this library's reading).  Row i of H_t
+// depends only on row i of H_{t-1}, on W and on the step's inputs:
+//   h_t = f_t h_{t-1} + (1 - f_t) tanh(h_{t-1} W + k_t[i] v_t),
+// so the rows of a pair are independent recurrences that share W and v_t.
+// The pages parallelise over batch × head with one matrix state per SM
+// (§2.2).  With few pairs that leaves most of the GPU idle, and the
+// tensor-core kernel's step is bound by its MMA round trip (issue, commit,
+// barrier wake-up: ~1,000 cycles), not by arithmetic.  This kernel instead
+// gives every state row its own warp: the row's vector-matrix product
+// h_{t-1}·W is 4,096 multiply-adds, which one warp does with W resident in
+// registers (lane l owns columns l and l + 32, so 64 fp32 pairs of W) as 64
+// packed FFMA2 instructions in four independent accumulator chains.  The only
+// exchange per step is the warp's own row through shared memory
+// (__syncwarp, no block barrier), so a step costs a few hundred cycles.
+//
+// Arithmetic: fp32 products of the fp32 state with W (bf16 values, exact in
+// fp32), fp32 sums in a fixed order, the same exp-based tanh as the
+// tensor-core kernel (or tanh.approx.f32 in the fast-tanh mode), the blend
+// h + (1 - f)(z - h).  This is more precise than the tensor-core kernel's
+// compensated bf16 operand, so the two kernels' states agree to rounding, not
+// bit for bit; within this kernel a row's result does not depend on the rest
+// of the batch or on how rows are grouped into CTAs.
+//
+// Layout: one CTA per (b, h) and slice of RS rows (RS warps), plus a bulk-copy
+// producer warp (this slice's RS values of k_t and q_t, the pair's v_t, f_t
+// for TC steps per ring stage) and a storer warp that sums the rows' readout
+// partials q_t[i]·h_t[i, :] in row order.  With several slices per pair the
+// slices' partial readouts go to the workspace and m2rnn_y_reduce_kernel adds
+// them in slice order.  Supported: V = 64 and RS = 8 rows per CTA: W takes 128
+// registers per lane, so an SM holds at most about 12 such warps, and at most
+// B·H·K/8 <= 148 CTAs (one wave, one CTA per SM).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace m2rnn {
+
+template <int RS_>
+struct FwdRowsCfg {
+    static constexpr int V = 64;
+    static constexpr int RS = RS_;                 // rows (warps) per CTA
+    static constexpr int TC = 16;                  // steps per ring stage
+    static constexpr int S = 4;                    // ring stages
+    static constexpr int W_PROD = RS, W_STORE = RS + 1;
+    static constexpr int NTHREADS = (RS + 2) * 32;
+    static constexpr int ST_K = 0;                 // [TC][RS] bf16
+    static constexpr int ST_Q = TC * RS * 2;       // [TC][RS] bf16
+    static constexpr int ST_V = 2 * TC * RS * 2;   // [TC][V] bf16
+    static constexpr int ST_F = ST_V + TC * V * 2; // [TC] fp32
+    static constexpr int STAGE_BYTES = ((ST_F + TC * 4) + 127) / 128 * 128;
+    static constexpr int YBUF_BYTES = TC * RS * V * 4;   // [TC][RS][V] readout partials
+    static constexpr int HROW_BYTES = 2 * V * 4;         // per warp: the row, double-buffered
+    static constexpr int OFF_RING = 0;
+    static constexpr int OFF_Y = OFF_RING + S * STAGE_BYTES;
+    static constexpr int OFF_H = OFF_Y + 2 * YBUF_BYTES;
+    static constexpr int OFF_BAR = OFF_H + RS * HROW_BYTES;
+    static constexpr int NBAR = 2 * S + 4;         // in_full, in_empty, ypfull[2], ypempty[2]
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
+    static_assert(RS == 8, "rows per CTA: the per-step k / q copies are RS·2 = 16 bytes, and W fills the registers");
+    static_assert(STAGE_BYTES % 128 == 0 && OFF_Y % 16 == 0 && OFF_H % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+    static_assert(SMEM_BYTES <= 227 * 1024, "smem");
+};
+
+template <int RS, bool FAST>
+__global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_kernel(const Params p) {
+    using C = FwdRowsCfg<RS>;
+    constexpr int V = C::V;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nsl = p.slices;
+    const int bh = blockIdx.x / nsl, sl = blockIdx.x % nsl;
+    const int K = p.K, koff = sl * RS;
+    const int hd = bh % p.H;
+    const int T = p.T;
+    const int nchunks = (T + C::TC - 1) / C::TC;
+    const int nck = (T + p.C - 1) / p.C;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    auto in_full = [&](int s) { return bar(s); };
+    auto in_empty = [&](int s) { return bar(C::S + s); };
+    auto ypfull = [&](int i) { return bar(2 * C::S + i); };
+    auto ypempty = [&](int i) { return bar(2 * C::S + 2 + i); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::NBAR);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::S; ++s) {
+            mbar_init(in_full(s), 1);
+            mbar_init(in_empty(s), RS);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(ypfull(i), RS);
+            mbar_init(ypempty(i), 1);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+
+    if (warp < RS) {
+        // ------------------------------------------------------------ one state row per warp
+        const int i = koff + warp;                 // state row of this warp
+        const int j0 = lane, j1 = lane + 32;       // state columns of this lane
+        // W columns j0, j1 as fp32 pairs, resident for all T steps
+        float2 Wr[V];
+        {
+            const uint16_t* Wg = static_cast<const uint16_t*>(p.W) + (size_t)hd * V * V;
+#pragma unroll
+            for (int l = 0; l < V; ++l)
+                Wr[l] = make_float2(bf16lo_to_f32(Wg[l * V + j0]), bf16lo_to_f32(Wg[l * V + j1]));
+        }
+        const size_t srow = ((size_t)bh * K + i) * V;   // row i of this pair's state
+        float2 h = p.H0 != nullptr ? make_float2(p.H0[srow + j0], p.H0[srow + j1]) : make_float2(0.f, 0.f);
+        if (p.ckpt != nullptr) {
+            float* ck = p.ckpt + (size_t)bh * nck * K * V + (size_t)i * V;
+            ck[j0] = h.x;
+            ck[j1] = h.y;
+        }
+        float* hrow = reinterpret_cast<float*>(smem + C::OFF_H + warp * C::HROW_BYTES);
+        bool ok = true;
+        for (int t = 0; t < T; ++t) {
+            const int c = t / C::TC, tt = t - c * C::TC, s = c % C::S;
+            const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            if (tt == 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (c / C::S) & 1, abort_flag, p));
+                if (ok && c >= 2)
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            // h_{t-1} to every lane of the warp.  The buffer alternates by step:
+            // every lane read this one at step t-2 before it reached the
+            // __syncwarp of step t-1, which this lane has passed.
+            float* hb = hrow + (t & 1) * V;
+            hb[j0] = h.x;
+            hb[j1] = h.y;
+            __syncwarp();
+            // a = h_{t-1}·W[:, (j0, j1)]: four accumulator chains over l mod 4
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+            const float4* hb4 = reinterpret_cast<const float4*>(hb);
+#pragma unroll
+            for (int l4 = 0; l4 < V / 4; ++l4) {
+                const float4 x = hb4[l4];
+                acc0 = __ffma2_rn(make_float2(x.x, x.x), Wr[4 * l4], acc0);
+                acc1 = __ffma2_rn(make_float2(x.y, x.y), Wr[4 * l4 + 1], acc1);
+                acc2 = __ffma2_rn(make_float2(x.z, x.z), Wr[4 * l4 + 2], acc2);
+                acc3 = __ffma2_rn(make_float2(x.w, x.w), Wr[4 * l4 + 3], acc3);
+            }
+            float2 a = __fadd2_rn(__fadd2_rn(acc0, acc1), __fadd2_rn(acc2, acc3));
+            const float ki = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_K + (tt * RS + warp) * 2));
+            const uint16_t* vt = reinterpret_cast<const uint16_t*>(st + C::ST_V + tt * V * 2);
+            a = __ffma2_rn(make_float2(ki, ki), make_float2(bf16lo_to_f32(vt[j0]), bf16lo_to_f32(vt[j1])), a);
+            const float z0 = FAST ? tanh_approx(a.x) : tanh_exp(a.x);
+            const float z1 = FAST ? tanh_approx(a.y) : tanh_exp(a.y);
+            const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
+            h = __ffma2_rn(make_float2(g, g), __fadd2_rn(make_float2(z0, z1), make_float2(-h.x, -h.y)), h);
+            // readout partial of this row: q_t[i]·h_t[i, :]
+            const float qi = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_Q + (tt * RS + warp) * 2));
+            float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * RS + warp) * V;
+            yb[j0] = qi * h.x;
+            yb[j1] = qi * h.y;
+            if (p.ckpt != nullptr && (t + 1) < T && ((t + 1) % p.C) == 0) {
+                float* ck = p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * K * V + (size_t)i * V;
+                ck[j0] = h.x;
+                ck[j1] = h.y;
+            }
+            if (tt == C::TC - 1 || t == T - 1) {
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(in_empty(s));
+                    mbar_arrive(ypfull(c & 1));
+                }
+            }
+        }
+        if (ok && p.HT != nullptr) {
+            p.HT[srow + j0] = h.x;
+            p.HT[srow + j1] = h.y;
+        }
+    } else if (warp == C::W_PROD) {
+        // ------------------------------------------------------------ producer
+        const int qkb = qk_pair(p, bh);   // k / q rows of this pair's head group
+        int last = -1;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % C::S;
+            if (p.fault == 1 && c >= 1) break;   // injected: stop feeding the ring after the first chunk
+            if (c >= C::S) {
+                const bool ok =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(in_empty(s), ((c / C::S) - 1) & 1, abort_flag, p));
+                if (!ok) break;
+            }
+            const int t0 = c * C::TC, nt = min(C::TC, T - t0);
+            uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
+            if (lane < nt)
+                reinterpret_cast<float*>(st + C::ST_F)[lane] = gate_value(p, p.f[(size_t)bh * T + t0 + lane]);
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t vb = (uint32_t)(nt * V * 2);
+                mbar_arrive_expect_tx(in_full(s), (uint32_t)(2 * nt * RS * 2) + vb);
+                bulk_g2s(smem_u32(st + C::ST_V), static_cast<const uint16_t*>(p.v) + ((size_t)bh * T + t0) * V, vb,
+                         in_full(s));
+            }
+            __syncwarp();
+            if (lane < nt) {   // this slice's RS values of each step's k and q row
+                const size_t r = ((size_t)qkb * T + t0 + lane) * K + koff;
+                bulk_g2s(smem_u32(st + C::ST_K + lane * RS * 2), static_cast<const uint16_t*>(p.k) + r, RS * 2,
+                         in_full(s));
+                bulk_g2s(smem_u32(st + C::ST_Q + lane * RS * 2), static_cast<const uint16_t*>(p.q) + r, RS * 2,
+                         in_full(s));
+            }
+            last = c;
+        }
+        // copies still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int c = max(0, last - C::S + 1); c <= last; ++c) mbar_wait_drain(in_full(c % C::S), (c / C::S) & 1, p);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ y storer
+        float* yout = nsl == 1 ? p.y : p.ypart + (size_t)sl * p.B * p.H * T * V;
+        for (int c = 0; c < nchunks; ++c) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(ypfull(c & 1), (c >> 1) & 1, abort_flag, p));
+            if (!ok) break;
+            const int t0 = c * C::TC, nt = min(C::TC, T - t0);
+            const float* yb = reinterpret_cast<const float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES);
+            float* yg = yout + ((size_t)bh * T + t0) * V;
+            for (int e = lane * 4; e < nt * V; e += 128) {
+                const int tt = e / V, jj = e % V;
+                const float* src = yb + tt * RS * V + jj;
+                float4 a = *reinterpret_cast<const float4*>(src);
+#pragma unroll
+                for (int r = 1; r < RS; ++r) {
+                    const float4 b = *reinterpret_cast<const float4*>(src + r * V);
+                    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+                }
+                *reinterpret_cast<float4*>(yg + e) = a;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ypempty(c & 1));
+        }
+    }
+}
+
+// Rows per CTA of the row kernel for B·H pairs of K x V states, or 0 when the
+// tensor-core kernel takes the problem: V = 64 and few enough rows that every
+// row gets a warp, 8 rows per CTA and one CTA per SM.
+int fwd_rows_per_cta(int B, int H, int K, int V) {
+    const long long pairs = (long long)B * H;
+    return (V == 64 && K % 8 == 0 && pairs * (K / 8) <= kNumSMs) ? 8 : 0;
+}
+
+template <int RS>
+static cudaError_t launch_rows(const Params& p0, cudaStream_t stream) {
+    using C = FwdRowsCfg<RS>;
+    Params p = p0;
+    p.slices = p.K / RS;
+    auto kern = p.fast_tanh ? m2rnn_fwd_rows_kernel<RS, true> : m2rnn_fwd_rows_kernel<RS, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<p.B * p.H * p.slices, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.slices == 1) return e;
+    return launch_y_reduce(p, stream);
+}
+
+cudaError_t launch_fwd_rows(const Params& p, cudaStream_t s) {
+    if (fwd_rows_per_cta(p.B, p.H, p.K, p.V) == 8) return launch_rows<8>(p, s);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace m2rnn

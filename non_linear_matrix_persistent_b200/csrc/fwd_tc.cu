@@ -442,19 +442,30 @@ __global__ void m2rnn_y_reduce_kernel(const Params p) {
     }
 }
 
-int fwd_tc_slices(int B, int H, int K) {
-    // Rows are split only while the (b, h) pairs alone would leave most SMs
-    // idle: a 16-row slice's step is ~1.45x shorter than a 64-row CTA's
-    // (measured on B200 at V = 64: ~1000 vs ~1430 cycles per step).
+int fwd_tc_slices(int B, int H, int K, int V) {
+    // Few pairs of 64-column states: the row kernel (fwd_rows.cu), 8 rows per CTA.
+    const int rs = fwd_rows_per_cta(B, H, K, V);
+    if (rs > 0) return K / rs;
+    // Otherwise rows are split only while the (b, h) pairs alone would leave
+    // most SMs idle: a 16-row slice's step is ~1.45x shorter than a 64-row
+    // CTA's (measured on B200 at V = 64: ~1000 vs ~1430 cycles per step).
     const long long pairs = (long long)B * H;
     int s = 1;
     while (s < 8 && K / (2 * s) >= 16 && pairs * 2 * s <= kNumSMs) s *= 2;
     return s;
 }
 
+cudaError_t launch_y_reduce(const Params& p, cudaStream_t s) {
+    const size_t n4 = (size_t)p.B * p.H * p.T * p.V / 4;
+    const int blocks = (int)((n4 + 255) / 256 < 1184 ? (n4 + 255) / 256 : 1184);
+    m2rnn_y_reduce_kernel<<<blocks, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_tc(const Params& p0, cudaStream_t s) {
+    if (fwd_rows_per_cta(p0.B, p0.H, p0.K, p0.V) > 0) return launch_fwd_rows(p0, s);
     Params p = p0;
-    p.slices = fwd_tc_slices(p.B, p.H, p.K);
+    p.slices = fwd_tc_slices(p.B, p.H, p.K, p.V);
     if (p.slices > 1) {
         cudaError_t e;
         switch (p.K / p.slices) {
@@ -464,10 +475,7 @@ cudaError_t launch_fwd_tc(const Params& p0, cudaStream_t s) {
             default: return cudaErrorInvalidValue;
         }
         if (e != cudaSuccess) return e;
-        const size_t n4 = (size_t)p.B * p.H * p.T * p.V / 4;
-        const int blocks = (int)((n4 + 255) / 256 < 1184 ? (n4 + 255) / 256 : 1184);
-        m2rnn_y_reduce_kernel<<<blocks, 256, 0, s>>>(p);
-        return cudaGetLastError();
+        return launch_y_reduce(p, s);
     }
     switch (p.K) {
         case 16: return launch_fwd_tc_k<16>(p, s);

@@ -63,13 +63,13 @@ size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward) {
         return 0;   // forward-only modes
     if (!backward && (d->mode == M2RNN_MODE_BF16_TC || d->mode == M2RNN_MODE_BF16_TC_FAST_TANH)) {
         // partial readouts of sliced rows
-        const int sl = m2rnn::fwd_tc_slices(d->B, d->H, d->K);
+        const int sl = m2rnn::fwd_tc_slices(d->B, d->H, d->K, d->V);
         if (sl > 1) n += sizeof(float) * (size_t)sl * d->B * d->H * d->T * d->V;
     }
     if (backward) {
         const size_t extra = d->mode == M2RNN_MODE_FP32_DEBUG
                                  ? m2rnn::bwd_fp32_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride)
-                                 : m2rnn::bwd_tc_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride);
+                                 : m2rnn::bwd_tc_workspace(d->B, d->H, d->T, d->K, d->V, d->ckpt_stride);
         n += (extra + 255) / 256 * 256;
         n += qk_group_partial_bytes(d);
     }
@@ -150,13 +150,13 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     p.dy = dy; p.dHT = dHT; p.dk = dk; p.dv = dv; p.dq = dq; p.df = df; p.dW = dW; p.dH0 = dH0;
     uint8_t* extra = static_cast<uint8_t*>(workspace) + kStatusBytes;
     p.dW_part = reinterpret_cast<float*>(extra);
-    p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K);
+    p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K, d->V);
     p.scratch = p.dW_part + (size_t)d->B * d->H * p.dw_parts * d->V * d->V;
     const bool grouped = qk_group_partial_bytes(d) != 0;
     if (grouped) {   // the kernels write per-head dk / dq here; the group sums go to dk, dq
         const size_t extra_bytes = d->mode == M2RNN_MODE_FP32_DEBUG
                                        ? m2rnn::bwd_fp32_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride)
-                                       : m2rnn::bwd_tc_workspace(d->B, d->H, d->K, d->V, d->ckpt_stride);
+                                       : m2rnn::bwd_tc_workspace(d->B, d->H, d->T, d->K, d->V, d->ckpt_stride);
         p.dk = reinterpret_cast<float*>(extra + (extra_bytes + 255) / 256 * 256);
         p.dq = p.dk + (size_t)d->B * d->H * d->T * d->K;
     }

@@ -33,8 +33,15 @@ def _dims(B=2, H=3, T=5, K=64, V=64, mode=0, C=16, G=0, logit=0):
 def test_workspace_size(L):
     # 128 (b, h) pairs fill the GPU: one CTA per pair, the forward needs only the status word
     assert L.m2rnn_workspace_size(_dims(B=8, H=16), 0) == 256
-    # 6 pairs: the forward splits the 64 rows into 4 slices and keeps their partial readouts
-    assert L.m2rnn_workspace_size(_dims(), 0) == 256 + 4 * (2 * 3 * 5 * 64) * 4
+    # 6 pairs of 64 x 64 states (384 rows <= 148 x 8): the row kernel, 8 rows
+    # per CTA, so 8 slices per pair whose partial readouts the workspace keeps
+    assert L.m2rnn_workspace_size(_dims(), 0) == 256 + 8 * (2 * 3 * 5 * 64) * 4
+    # 16 pairs of 64 x 64 (1024 rows): still the row kernel; 32 pairs (2048 rows): the
+    # tensor-core kernel with 4 slices of 16 rows
+    assert L.m2rnn_workspace_size(_dims(B=1, H=16), 0) == 256 + 8 * (16 * 5 * 64) * 4
+    assert L.m2rnn_workspace_size(_dims(B=2, H=16), 0) == 256 + 4 * (32 * 5 * 64) * 4
+    # other widths take the tensor-core kernel: 6 pairs split the 64 rows into 4 slices
+    assert L.m2rnn_workspace_size(_dims(V=32), 0) == 256 + 4 * (2 * 3 * 5 * 32) * 4
     assert L.m2rnn_workspace_size(_dims(mode=1), 0) == 256   # fp32 debug mode: no slices
     assert L.m2rnn_workspace_size(_dims(mode=1), 1) > 256
     assert L.m2rnn_workspace_size(_dims(K=48), 0) == 0
@@ -91,6 +98,30 @@ def test_backward_argument_errors(L):
     # the fast-tanh and register-resident modes are forward only
     assert bwd(_dims(mode=_lib.MODE_BF16_TC_FAST_TANH)) == _lib.ERR_INVALID_ARG
     assert bwd(_dims(mode=_lib.MODE_BF16_MMA_SYNC)) == _lib.ERR_INVALID_ARG
+
+
+def test_tc_backward_every_shape_has_a_workspace(L):
+    """The tensor-core backward takes every K, V in {16, 32, 64, 128} with a
+    checkpoint stride of at most 16.  V = 64 with K >= 32 keeps the
+    extended-operand kernel's workspace (dW partials + 2·C·K·V scratch per
+    pair); K = 128 at V = 128 runs four 32-row slices per pair, whose dv and
+    df partials (4·B·H·T·(V + 1) fp32) are summed after the kernel."""
+    B, H, T, C = 2, 3, 5, 4
+    for K in (16, 32, 64, 128):
+        for V in (16, 32, 64, 128):
+            assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=K, V=V, C=C), 1) > 256, (K, V)
+            # a longer stride gets only the status word, and the call is rejected before any launch
+            assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=K, V=V, C=17), 1) == 256, (K, V)
+            st = L.m2rnn_backward(_dims(B=B, H=H, T=T, K=K, V=V, C=17), *([4096] * 7), None, *([4096] * 7),
+                                  1 << 40, None)
+            assert st == _lib.ERR_UNSUPPORTED_SHAPE, (K, V)
+    def pad(n):
+        return 256 + (n + 255) // 256 * 256
+    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=64, V=64, C=C), 1) == pad(
+        4 * (B * H * 64 * 64 + B * H * 2 * C * 64 * 64))
+    ncta = B * H * 4
+    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=128, V=128, C=C), 1) == pad(
+        4 * (ncta * 128 * 128 + 2 * C * ncta * 32 * 128 + 4 * B * H * T * 129))
 
 
 def test_fast_tanh_mode_workspace(L):

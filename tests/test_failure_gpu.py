@@ -16,10 +16,12 @@ from oracle import oracle
 pytestmark = pytest.mark.gpu
 
 
-def test_injected_stall_reports_timeout_and_context_stays_usable():
+@pytest.mark.parametrize("V", [64, 32])
+def test_injected_stall_reports_timeout_and_context_stays_usable(V):
+    """V = 64 with 4 pairs runs the row kernel, V = 32 the tensor-core kernel."""
     from non_linear_matrix_persistent_b200 import _lib, api
     L = _lib.lib()
-    w = Workload("stall", B=2, H=2, T=40, K=64, V=64, h0_range=0.5, seed=4)
+    w = Workload("stall", B=2, H=2, T=40, K=64, V=V, h0_range=0.5, seed=4)
     x = make_inputs(w)
     xc = {n: (None if t is None else t.cuda()) for n, t in x.items()}
     api.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"])   # creates the workspace

@@ -206,21 +206,55 @@ def test_tc_batch_independence_bitwise():
 
 @pytest.mark.parametrize("K", [64, 128])
 def test_row_slices_match_whole_rows(K):
-    """Few (b, h) pairs: the forward splits each pair's rows over several CTAs
-    (rows of H are independent) and sums their partial readouts.  The states
-    must equal the one-CTA-per-pair result bit for bit; y differs only in the
-    order of the readout sum."""
+    """Few (b, h) pairs: the tensor-core forward splits each pair's rows over
+    several CTAs (rows of H are independent) and sums their partial readouts.
+    The states must equal the one-CTA-per-pair result bit for bit; y differs
+    only in the order of the readout sum.  (V = 32: at V = 64 few pairs run the
+    row kernel instead.)"""
     from non_linear_matrix_persistent_b200 import _lib
-    big = Workload("rs", B=8, H=16, T=37, K=K, V=64, h0_range=0.5, seed=9)
-    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(8, 16, 37, K, 64, 0, 16), 0) == 256   # one CTA per pair
+    big = Workload("rs", B=8, H=16, T=37, K=K, V=32, h0_range=0.5, seed=9)
+    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(8, 16, 37, K, 32, 0, 16), 0) == 256   # one CTA per pair
     xc = _cuda(make_inputs(big))
     y, HT, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=8, want_ckpt=True)
     s = {n: (None if t is None else t[3:4].contiguous()) for n, t in xc.items() if n != "W"}
-    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(1, 16, 37, K, 64, 0, 16), 0) > 256   # sliced rows
+    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(1, 16, 37, K, 32, 0, 16), 0) > 256   # sliced rows
     y1, HT1, ck1 = api().forward(s["k"], s["v"], s["q"], s["f"], xc["W"], s["H0"], ckpt_stride=8, want_ckpt=True)
     torch.cuda.synchronize()
     assert torch.equal(HT[3:4], HT1) and torch.equal(ck[3:4], ck1)
     assert torch.allclose(y[3:4], y1, rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("K", [16, 64])
+def test_row_kernel_agrees_with_tensor_core_kernel(K):
+    """Few pairs of 64-column states (at most 148 CTAs of 8 rows) run the row
+    kernel (one warp per state row, fp32 FFMA); a full batch runs the
+    tensor-core kernel (compensated bf16 operand).  On the same pairs the two
+    agree to rounding and both are within the tensor-core tolerance of the
+    oracle; the row kernel's states and y do not depend on the rest of the
+    batch, bit for bit."""
+    from non_linear_matrix_persistent_b200 import _lib
+    B, H, T = 8, 16, 45
+    big = Workload("rk", B=B, H=H, T=T, K=K, V=64, h0_range=0.5, seed=13)
+    x = make_inputs(big)
+    xc = _cuda(x)
+    assert _lib.lib().m2rnn_workspace_size(_lib.Dims(B, H, T, K, 64, 0, 16), 0) == 256   # tensor cores
+    y, HT, _ = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"])
+    outs = []
+    for nh in (H, H // 2):   # batch row 3 with all heads, then with the first half of them
+        s = {n: (None if t is None else t[3:4, :nh].contiguous()) for n, t in xc.items() if n != "W"}
+        assert _lib.lib().m2rnn_workspace_size(_lib.Dims(1, nh, T, K, 64, 0, 16), 0) == \
+            256 + (K // 8) * nh * T * 64 * 4   # row kernel, 8 rows per CTA
+        y1, HT1, _ = api().forward(s["k"], s["v"], s["q"], s["f"], xc["W"][:nh].contiguous(), s["H0"])
+        outs.append((y1[0], HT1[0]))
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    half = H // 2
+    assert torch.equal(outs[0][0][:half], outs[1][0]) and torch.equal(outs[0][1][:half], outs[1][1])
+    y1, HT1 = outs[0]
+    assert float((HT1 - HT[3]).abs().max()) <= 1e-4 and float((y1 - y[3]).abs().max()) <= 1e-4
+    sel = {n: (None if t is None else t[3:4]) for n, t in x.items() if n != "W"}
+    yr, HTr = oracle.forward(sel["k"], sel["v"], sel["q"], sel["f"], x["W"], sel["H0"])
+    _check_fwd("row_kernel_K%d" % K, y1[None], HT1[None], yr, HTr, "bf16")
 
 
 @pytest.mark.parametrize("mode,K,V", [("bf16", 64, 64), ("bf16", 128, 32), ("fp32", 32, 16)])
@@ -344,14 +378,60 @@ def test_fp32_backward_small(K, V, T, C):
     _check_grads("fp32_bwd_K%d_V%d_T%d_C%d" % (K, V, T, C), g, gr, 1e-4)
 
 
-def test_tc_backward_unsupported_shape():
+def test_tc_backward_unsupported_checkpoint_stride():
+    """The tensor-core backward keeps at most 16 steps of a chunk on chip."""
     from non_linear_matrix_persistent_b200._lib import ERR_UNSUPPORTED_SHAPE, M2RNNError
-    w = Workload("u", B=1, H=1, T=4, K=64, V=128, backward=True)
+    w = Workload("u", B=1, H=1, T=40, K=64, V=128, backward=True)
     xc = _cuda(make_inputs(w))
-    _, _, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=4, want_ckpt=True)
+    _, _, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=17, want_ckpt=True)
     with pytest.raises(M2RNNError) as e:
-        api().backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=4)
+        api().backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=17)
     assert e.value.status == ERR_UNSUPPORTED_SHAPE
+
+
+@pytest.mark.parametrize("K,V", [(k, v) for k in (16, 32, 64, 128) for v in (16, 32, 64, 128)])
+@pytest.mark.parametrize("T,C", [(1, 16), (17, 8), (40, 16), (33, 5)])
+@pytest.mark.parametrize("with_dHT", [False, True])
+def test_tc_backward_every_shape(K, V, T, C, with_dHT):
+    """Every K, V in {16, 32, 64, 128} on the tensor cores: V = 64 with K >= 32
+    runs the extended-operand kernel, the rest the general-shape kernel (K = 128
+    at V = 128 as four 32-row slices whose dv and df are summed in order)."""
+    w = Workload("bwall", B=2, H=3, T=T, K=K, V=V, h0_range=0.5, backward=True, seed=K + 3 * V + T + C)
+    x = make_inputs(w)
+    dHT = torch.randn(2, 3, K, V, generator=torch.Generator().manual_seed(8)) if with_dHT else None
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, C, None if dHT is None else dHT.cuda())
+    gr = _oracle_bwd(x, dHT)
+    _check_grads("tc_bwd_all_K%d_V%d_T%d_C%d_dHT%d" % (K, V, T, C, int(with_dHT)), g, gr, GRAD_REL)
+
+
+@pytest.mark.parametrize("K,V,G,logit", [(128, 128, 2, False), (32, 16, 0, True), (16, 64, 1, True),
+                                         (64, 32, 2, True), (128, 128, 0, True)])
+def test_tc_backward_general_shapes_grouped_and_logit(K, V, G, logit):
+    """Grouped k / q and gate logits through the general-shape backward."""
+    w = Workload("gsh", B=2, H=4, T=37, K=K, V=V, h0_range=0.5, backward=True, qk_heads=G, gate_logits=logit,
+                 gate_var=4.0 if logit else 1.0, seed=K + V + G)
+    x = make_inputs(w)
+    xc = _cuda(x)
+    a = api()
+    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=8, want_ckpt=True,
+                         f_is_logit=logit)
+    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=8, f_is_logit=logit)
+    torch.cuda.synchronize()
+    assert a.device_status() == 0
+    gr = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], f_is_logit=logit)
+    _check_grads("gen_bwd_K%d_V%d_G%d_logit%d" % (K, V, G, int(logit)), g, gr, GRAD_REL)
+
+
+def test_tc_backward_general_shapes_deterministic():
+    """Two runs of the general-shape backward (four slices per pair) give the
+    same bits: every sum, the slices' included, runs in a fixed order."""
+    w = Workload("det", B=2, H=2, T=45, K=128, V=128, h0_range=0.5, backward=True, seed=3)
+    xc = _cuda(make_inputs(w))
+    g1 = {n: t.clone() for n, t in _gpu_fwd_bwd(xc, 8).items()}
+    g2 = _gpu_fwd_bwd(xc, 8)
+    for n in g1:
+        assert torch.equal(g1[n], g2[n]), n
 
 
 def test_train_workload_sampled_head():
@@ -370,6 +450,29 @@ def test_train_workload_sampled_head():
     gr = _oracle_bwd(sel)
     gs = {n: (t[:, h:h + 1] if n != "dW" else t[h:h + 1]) for n, t in g.items()}
     _check_grads("full_layer410m_train_head%d" % h, gs, gr, GRAD_REL)
+
+
+def test_train_7b_moe_shape_sampled_head():
+    """The 7B-MoE layer shape trained (B=4, H=32, K=V=128, T=4096; forward with
+    checkpoints every 16 steps, then the general-shape backward) in the
+    launch configuration the benchmark times; the oracle checks one whole head
+    (all four batch rows, so dW[h] is complete), pair by pair."""
+    w = WORKLOADS["layer7b_moe_train"]
+    x = make_inputs(w)
+    xc = _cuda(x)
+    g = _gpu_fwd_bwd(xc, 16)
+    for n, t in g.items():
+        assert torch.isfinite(t).all(), n
+    h = 11
+    sel = {n: (None if t is None else t[:, h:h + 1].contiguous()) for n, t in x.items() if n != "W"}
+    sel["W"] = x["W"][h:h + 1].contiguous()
+    gr = _oracle_bwd(sel)
+    gs = {n: (t[:, h:h + 1] if n != "dW" else t[h:h + 1]) for n, t in g.items()}
+    _check_grads("full_layer7b_moe_train_head%d" % h, gs, gr, GRAD_REL)
+    for b in range(w.B):   # each pair on its own
+        _check_grads("full_layer7b_moe_train_b%d" % b,
+                     {n: (t[b:b + 1] if n != "dW" else gr["dW"]) for n, t in gs.items()},
+                     {n: (r[b:b + 1] if n != "dW" else r) for n, r in gr.items()}, GRAD_REL)
 
 
 # ---------------------------------------------------------------- grouped k / q
