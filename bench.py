@@ -140,6 +140,33 @@ def per_step_counts(w):
     return fwd, bwd
 
 
+def forward_kernel(w):
+    """(kernel name, source file) of the forward that runs for workload w, by
+    the library's dispatch rule: the fp32 debug mode has its own kernel;
+    64-column states with B·H·K/8 <= 148 rows-of-8 run the row kernel (one
+    warp per state row); everything else the tcgen05 kernel."""
+    if w.mode != "bf16":
+        return "m2rnn_fwd_fp32_kernel", "debug_fp32.cu"
+    if w.V == 64 and w.K % 8 == 0 and w.B * w.H * (w.K // 8) <= NUM_SMS:
+        return "m2rnn_fwd_rows_kernel", "fwd_rows.cu"
+    return "m2rnn_fwd_tc_kernel", "fwd_tc.cu"
+
+
+def backward_kernel(w):
+    """(kernel name, source file) of the tensor-core backward for workload w:
+    the extended-operand kernel for V = 64 with K >= 32, the general-shape
+    kernel otherwise."""
+    if w.V == 64 and w.K in (32, 64, 128):
+        return "m2rnn_bwd_tc_kernel", "bwd_tc.cu"
+    return "m2rnn_bwd_tcg_kernel", "bwd_tcg.cu"
+
+
+def profile_name(kernel, workload):
+    """profiles/ summary of one kernel on one workload: m2rnn_fwd_tc_kernel on
+    layer410m_train is m2rnn_fwd_tc_layer410m_train.md."""
+    return "%s_%s.md" % (kernel[:-len("_kernel")], workload)
+
+
 def launches_per_step(w) -> int:
     """Kernels of this library that one step launches: the forward scan, plus
     the sum of the row slices' partial readouts when the forward splits rows
@@ -165,8 +192,9 @@ def kernel_digest(src: bytes) -> str:
     return hashlib.sha256((code + "\n" + flags).encode()).hexdigest()[:16]
 
 
-# Headers every kernel file includes; a profile is tied to them as well.
-KERNEL_HEADERS = ("common.cuh", "ptx.cuh", "tc_common.cuh", "kernels.h")
+# Device-code headers the kernel files include; a profile is tied to them as
+# well (kernels.h holds only host-side declarations).
+KERNEL_HEADERS = ("common.cuh", "ptx.cuh", "tc_common.cuh")
 
 
 def kernel_source(kernel_file: str) -> bytes:
@@ -228,7 +256,11 @@ def _oracle_sample(w, pairs, cores):
     return run
 
 
-def kernel_entry(ms_mean, cnt, units, T, peaks, peak_kind, sm_max, sm_mhz, tanh_kind="accurate", traffic=None):
+FMA_PER_SM_PER_CLK = 128     # fp32 fused multiply-adds per SM per clock (CUDA cores)
+
+
+def kernel_entry(ms_mean, cnt, units, T, peaks, peak_kind, sm_max, sm_mhz, tanh_kind="accurate", traffic=None,
+                 pipe="tensor"):
     """Roofline figures of one kernel from its mean CUDA-event time.
 
     The bound is the special-function unit: the method evaluates one tanh per
@@ -236,7 +268,10 @@ def kernel_entry(ms_mean, cnt, units, T, peaks, peak_kind, sm_max, sm_mhz, tanh_
     148 SMs x 16 results per SM per clock x the maximum SM clock.  The SFU
     operations the implementation spends per tanh are reported apart
     (`sfu_ops`); the tensor-pipe and HBM fractions of the same launch go beside
-    them.  `units` is the (b, h, t) steps one launch processes."""
+    them.  `units` is the (b, h, t) steps one launch processes.  `pipe` names
+    where the transition product runs: "tensor" (tcgen05 or mma.sync, against
+    the measured bf16 peak) or "fma" (CUDA-core FFMA, against the derived fp32
+    peak 148 SMs x 128 FMA x 2 FLOP x the maximum SM clock)."""
     s = ms_mean / 1e3
     tanh_rate = cnt["tanh"] * units / s / 1e9
     sfu_peak = NUM_SMS * SFU_PER_SM_PER_CLK * sm_max * 1e6 / 1e9
@@ -256,9 +291,18 @@ def kernel_entry(ms_mean, cnt, units, T, peaks, peak_kind, sm_max, sm_mhz, tanh_
     }
     if cnt.get("flop"):
         tf = cnt["flop"] * units / s / 1e12
-        e["tensor"] = {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
-                       "frac": tf / peaks["bf16_tflops"], "peak_kind": peak_kind}
+        if pipe == "tensor":
+            e["tensor"] = {"achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
+                           "frac": tf / peaks["bf16_tflops"], "peak_kind": peak_kind}
+        else:
+            fpk = NUM_SMS * FMA_PER_SM_PER_CLK * 2 * sm_max * 1e6 / 1e12
+            e["fma"] = {"achieved_tflops": tf, "peak_tflops": fpk, "frac": tf / fpk, "peak_kind": "derived"}
     return e
+
+
+def kernel_pipe(kernel):
+    """Where a kernel's transition product runs (see kernel_entry)."""
+    return "fma" if kernel in ("m2rnn_fwd_rows_kernel", "m2rnn_fwd_fp32_kernel") else "tensor"
 
 
 def time_forward_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_max, sm_mhz):
@@ -290,10 +334,10 @@ def time_forward_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_ma
             raise RuntimeError("device-side wait ran out in the %s forward" % name)
         ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
         cnt, _ = per_step_counts(w)
-        if w.mode != "bf16":
-            cnt = dict(cnt, flop=0.0)   # the fp32 debug mode runs on CUDA cores
-        traffic = measured_traffic("fwd_tc.cu", "m2rnn_fwd_tc_%s.md" % name) if kind == "accurate" else None
-        e = kernel_entry(ms, cnt, B * H * T, T, peaks, peak_kind, sm_max, sm_mhz, kind, traffic)
+        kname, ksrc = forward_kernel(w)
+        traffic = measured_traffic(ksrc, profile_name(kname, name)) if kind == "accurate" else None
+        e = kernel_entry(ms, cnt, B * H * T, T, peaks, peak_kind, sm_max, sm_mhz, kind, traffic, kernel_pipe(kname))
+        e["kernel"] = kname
         e["tokens_per_s"] = B * T / (ms / 1e3)
         e["steps"] = steps
         res["forward" if kind == "accurate" else "forward_fast_tanh"] = e
@@ -340,8 +384,12 @@ def time_training_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_m
     units = B * H * T
     res = {"B": B, "H": H, "T": T, "K": K, "V": V, "ckpt_stride": C, "tokens": B * T, "steps": steps,
            "ms_per_step": fwd + bwd, "tokens_per_s": B * T / ((fwd + bwd) / 1e3),
-           "forward": kernel_entry(fwd, cf, units, T, peaks, peak_kind, sm_max, sm_mhz),
+           "forward": kernel_entry(fwd, cf, units, T, peaks, peak_kind, sm_max, sm_mhz,
+                                   pipe=kernel_pipe(forward_kernel(w)[0])),
            "backward": kernel_entry(bwd, cb, units, T, peaks, peak_kind, sm_max, sm_mhz)}
+    for part, (kname, ksrc) in (("forward", forward_kernel(w)), ("backward", backward_kernel(w))):
+        res[part]["kernel"] = kname
+        res[part]["traffic"] = measured_traffic(ksrc, profile_name(kname, name))
     del x, out, gout
     return res
 
@@ -545,13 +593,13 @@ def main():
     cf, cb = per_step_counts(w)
     units = B * H * T   # (b, h, t) steps per launch on this rank
     kernels = {}
-    for name, ms_list, cnt, src, prof in (
-            ("m2rnn_fwd_tc_kernel", fwd_ms, cf, "fwd_tc.cu", "m2rnn_fwd_tc_%s.md" % w.name),
-            ("m2rnn_bwd_tc_kernel", bwd_ms, cb, "bwd_tc.cu", "m2rnn_bwd_tc_%s.md" % w.name)):
-        if name.startswith("m2rnn_bwd") and not w.backward:
+    for (name, src), ms_list, cnt, bwd in ((forward_kernel(w), fwd_ms, cf, False),
+                                          (backward_kernel(w), bwd_ms, cb, True)):
+        if bwd and not w.backward:
             continue
         kernels[name] = kernel_entry(statistics.mean(ms_list), cnt, units, T, peaks, peak_kind, sm_max, sm_mhz,
-                                     "accurate", measured_traffic(src, prof))
+                                     "accurate", measured_traffic(src, profile_name(name, w.name)),
+                                     kernel_pipe(name))
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
     roofline = dict(kernel=dom, **{k: v for k, v in kernels[dom].items()})
     roofline["kernels"] = kernels

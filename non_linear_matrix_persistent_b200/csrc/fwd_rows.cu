@@ -1,4 +1,4 @@
-// M²RNN forward scan for few (b, h) pairs: one warp per state row, CUDA-core
+// M²RNN forward scan for few (b, h) pairs: two state rows per warp, CUDA-core
 // FFMA, no per-step barrier.
 //
 // Recurrence (gist.science technical summary of "M²RNN: Non-Linear RNNs with
@@ -11,13 +11,18 @@
 // The pages parallelise over batch × head with one matrix state per SM
 // (§2.2).  With few pairs that leaves most of the GPU idle, and the
 // tensor-core kernel's step is bound by its MMA round trip (issue, commit,
-// barrier wake-up: ~1,000 cycles), not by arithmetic.  This kernel instead
-// gives every state row its own warp: the row's vector-matrix product
-// h_{t-1}·W is 4,096 multiply-adds, which one warp does with W resident in
-// registers (lane l owns columns l and l + 32, so 64 fp32 pairs of W) as 64
-// packed FFMA2 instructions in four independent accumulator chains.  The only
-// exchange per step is the warp's own row through shared memory
-// (__syncwarp, no block barrier), so a step costs a few hundred cycles.
+// barrier wake-up: ~1,000 cycles), not by arithmetic.  This kernel gives each
+// warp two state rows for all T steps instead, with W resident in registers,
+// so a step needs no block-level synchronisation at all: the warp shares its
+// two rows through shared memory (__syncwarp), every lane reads both rows in
+// 16-byte broadcast loads, and lane l forms columns l and l + 32 of each row's
+// product h_{t-1}·W with packed FFMA2 (W[l'][l], W[l'][l + 32] as fp32 pairs,
+// 64 of them, shared by the two rows) in four accumulator chains per row.
+// Measured on B200 at the long B = 1 workload (1,024 rows on 128 SMs): one
+// row per warp 8.1 ms, two rows per warp (this kernel) 6.2 ms; slower were
+// the same with the h row stored as duplicated pairs (7.9 ms), a row pair
+// split over two warps by columns (8.5 ms) and a two-dimensional split of the
+// product over the lanes with a shuffle reduce-scatter (8.1 / 8.7 ms).
 //
 // Arithmetic: fp32 products of the fp32 state with W (bf16 values, exact in
 // fp32), fp32 sums in a fixed order, the same exp-based tanh as the
@@ -27,14 +32,13 @@
 // bit for bit; within this kernel a row's result does not depend on the rest
 // of the batch or on how rows are grouped into CTAs.
 //
-// Layout: one CTA per (b, h) and slice of RS rows (RS warps), plus a bulk-copy
-// producer warp (this slice's RS values of k_t and q_t, the pair's v_t, f_t
-// for TC steps per ring stage) and a storer warp that sums the rows' readout
-// partials q_t[i]·h_t[i, :] in row order.  With several slices per pair the
-// slices' partial readouts go to the workspace and m2rnn_y_reduce_kernel adds
-// them in slice order.  Supported: V = 64 and RS = 8 rows per CTA: W takes 128
-// registers per lane, so an SM holds at most about 12 such warps, and at most
-// B·H·K/8 <= 148 CTAs (one wave, one CTA per SM).
+// Layout: one CTA per (b, h) and slice of RS = 8 rows (4 row warps), plus a
+// bulk-copy producer warp (this slice's 8 values of k_t and q_t, the pair's
+// v_t, f_t for TC steps per ring stage) and a storer warp that sums the rows'
+// readout partials q_t[i]·h_t[i, :] in row order.  With several slices per
+// pair the slices' partial readouts go to the workspace and
+// m2rnn_y_reduce_kernel adds them in slice order.  Supported: V = 64 (W takes
+// 128 registers per lane) and at most 148 CTAs (one wave, one CTA per SM).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -46,25 +50,27 @@ namespace m2rnn {
 template <int RS_>
 struct FwdRowsCfg {
     static constexpr int V = 64;
-    static constexpr int RS = RS_;                 // rows (warps) per CTA
+    static constexpr int RS = RS_;                 // rows per CTA
+    static constexpr int RW = 2;                   // rows per warp (sharing the W registers)
+    static constexpr int NWR = RS / RW;            // row warps
     static constexpr int TC = 16;                  // steps per ring stage
     static constexpr int S = 4;                    // ring stages
-    static constexpr int W_PROD = RS, W_STORE = RS + 1;
-    static constexpr int NTHREADS = (RS + 2) * 32;
+    static constexpr int W_PROD = NWR, W_STORE = NWR + 1;
+    static constexpr int NTHREADS = (NWR + 2) * 32;
     static constexpr int ST_K = 0;                 // [TC][RS] bf16
     static constexpr int ST_Q = TC * RS * 2;       // [TC][RS] bf16
     static constexpr int ST_V = 2 * TC * RS * 2;   // [TC][V] bf16
     static constexpr int ST_F = ST_V + TC * V * 2; // [TC] fp32
     static constexpr int STAGE_BYTES = ((ST_F + TC * 4) + 127) / 128 * 128;
     static constexpr int YBUF_BYTES = TC * RS * V * 4;   // [TC][RS][V] readout partials
-    static constexpr int HROW_BYTES = 2 * V * 4;         // per warp: the row, double-buffered
+    static constexpr int HROW_BYTES = 2 * RW * V * 4;    // per warp: its rows, double-buffered
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_Y = OFF_RING + S * STAGE_BYTES;
     static constexpr int OFF_H = OFF_Y + 2 * YBUF_BYTES;
-    static constexpr int OFF_BAR = OFF_H + RS * HROW_BYTES;
+    static constexpr int OFF_BAR = OFF_H + NWR * HROW_BYTES;
     static constexpr int NBAR = 2 * S + 4;         // in_full, in_empty, ypfull[2], ypempty[2]
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
-    static_assert(RS == 8, "rows per CTA: the per-step k / q copies are RS·2 = 16 bytes, and W fills the registers");
+    static_assert(RS == 8, "rows per CTA: the per-step k / q copies are RS·2 = 16 bytes");
     static_assert(STAGE_BYTES % 128 == 0 && OFF_Y % 16 == 0 && OFF_H % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
@@ -94,10 +100,10 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::S; ++s) {
             mbar_init(in_full(s), 1);
-            mbar_init(in_empty(s), RS);
+            mbar_init(in_empty(s), C::NWR);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(ypfull(i), RS);
+            mbar_init(ypfull(i), C::NWR);
             mbar_init(ypempty(i), 1);
         }
         *abort_flag = 0;
@@ -105,9 +111,10 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
     }
     __syncthreads();
 
-    if (warp < RS) {
-        // ------------------------------------------------------------ one state row per warp
-        const int i = koff + warp;                 // state row of this warp
+    if (warp < C::NWR) {
+        // ------------------------------------------------------------ two state rows per warp
+        const int r0 = warp * 2;                   // first row of this warp within the slice
+        const int i = koff + r0;                   // its state row
         const int j0 = lane, j1 = lane + 32;       // state columns of this lane
         // W columns j0, j1 as fp32 pairs, resident for all T steps
         float2 Wr[V];
@@ -117,12 +124,12 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             for (int l = 0; l < V; ++l)
                 Wr[l] = make_float2(bf16lo_to_f32(Wg[l * V + j0]), bf16lo_to_f32(Wg[l * V + j1]));
         }
-        const size_t srow = ((size_t)bh * K + i) * V;   // row i of this pair's state
-        float2 h = p.H0 != nullptr ? make_float2(p.H0[srow + j0], p.H0[srow + j1]) : make_float2(0.f, 0.f);
+        const size_t srow0 = ((size_t)bh * K + i) * V, srow1 = srow0 + V;
+        float2 h0 = p.H0 != nullptr ? make_float2(p.H0[srow0 + j0], p.H0[srow0 + j1]) : make_float2(0.f, 0.f);
+        float2 h1 = p.H0 != nullptr ? make_float2(p.H0[srow1 + j0], p.H0[srow1 + j1]) : make_float2(0.f, 0.f);
         if (p.ckpt != nullptr) {
             float* ck = p.ckpt + (size_t)bh * nck * K * V + (size_t)i * V;
-            ck[j0] = h.x;
-            ck[j1] = h.y;
+            ck[j0] = h0.x; ck[j1] = h0.y; ck[V + j0] = h1.x; ck[V + j1] = h1.y;
         }
         float* hrow = reinterpret_cast<float*>(smem + C::OFF_H + warp * C::HROW_BYTES);
         bool ok = true;
@@ -136,41 +143,58 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
                                     mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
                 if (!ok) break;
             }
-            // h_{t-1} to every lane of the warp.  The buffer alternates by step:
+            // both rows of h_{t-1} to every lane.  The buffer alternates by step:
             // every lane read this one at step t-2 before it reached the
             // __syncwarp of step t-1, which this lane has passed.
-            float* hb = hrow + (t & 1) * V;
-            hb[j0] = h.x;
-            hb[j1] = h.y;
+            float* hb = hrow + (t & 1) * 2 * V;
+            hb[j0] = h0.x; hb[j1] = h0.y; hb[V + j0] = h1.x; hb[V + j1] = h1.y;
             __syncwarp();
-            // a = h_{t-1}·W[:, (j0, j1)]: four accumulator chains over l mod 4
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+            const uint32_t kk = *reinterpret_cast<const uint32_t*>(st + C::ST_K + (tt * RS + r0) * 2);
+            const uint16_t* vt = reinterpret_cast<const uint16_t*>(st + C::ST_V + tt * V * 2);
+            const float2 v2 = make_float2(bf16lo_to_f32(vt[j0]), bf16lo_to_f32(vt[j1]));
+            // h_{t-1}·W[:, (j0, j1)] for both rows: four accumulator chains per row over l mod 4
+            float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0, b0 = a0, b1 = a0, b2 = a0, b3 = a0;
             const float4* hb4 = reinterpret_cast<const float4*>(hb);
 #pragma unroll
-            for (int l4 = 0; l4 < V / 4; ++l4) {
-                const float4 x = hb4[l4];
-                acc0 = __ffma2_rn(make_float2(x.x, x.x), Wr[4 * l4], acc0);
-                acc1 = __ffma2_rn(make_float2(x.y, x.y), Wr[4 * l4 + 1], acc1);
-                acc2 = __ffma2_rn(make_float2(x.z, x.z), Wr[4 * l4 + 2], acc2);
-                acc3 = __ffma2_rn(make_float2(x.w, x.w), Wr[4 * l4 + 3], acc3);
+            for (int b = 0; b < V / 4; b += 4) {
+                float4 xs[4], ys[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) { xs[u] = hb4[b + u]; ys[u] = hb4[V / 4 + b + u]; }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int l4 = b + u;
+                    a0 = __ffma2_rn(make_float2(xs[u].x, xs[u].x), Wr[4 * l4], a0);
+                    b0 = __ffma2_rn(make_float2(ys[u].x, ys[u].x), Wr[4 * l4], b0);
+                    a1 = __ffma2_rn(make_float2(xs[u].y, xs[u].y), Wr[4 * l4 + 1], a1);
+                    b1 = __ffma2_rn(make_float2(ys[u].y, ys[u].y), Wr[4 * l4 + 1], b1);
+                    a2 = __ffma2_rn(make_float2(xs[u].z, xs[u].z), Wr[4 * l4 + 2], a2);
+                    b2 = __ffma2_rn(make_float2(ys[u].z, ys[u].z), Wr[4 * l4 + 2], b2);
+                    a3 = __ffma2_rn(make_float2(xs[u].w, xs[u].w), Wr[4 * l4 + 3], a3);
+                    b3 = __ffma2_rn(make_float2(ys[u].w, ys[u].w), Wr[4 * l4 + 3], b3);
+                }
             }
-            float2 a = __fadd2_rn(__fadd2_rn(acc0, acc1), __fadd2_rn(acc2, acc3));
-            const float ki = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_K + (tt * RS + warp) * 2));
-            const uint16_t* vt = reinterpret_cast<const uint16_t*>(st + C::ST_V + tt * V * 2);
-            a = __ffma2_rn(make_float2(ki, ki), make_float2(bf16lo_to_f32(vt[j0]), bf16lo_to_f32(vt[j1])), a);
-            const float z0 = FAST ? tanh_approx(a.x) : tanh_exp(a.x);
-            const float z1 = FAST ? tanh_approx(a.y) : tanh_exp(a.y);
+            float2 A0 = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+            float2 A1 = __fadd2_rn(__fadd2_rn(b0, b1), __fadd2_rn(b2, b3));
+            const float k0 = bf16lo_to_f32(kk), k1 = bf16hi_to_f32(kk);
+            A0 = __ffma2_rn(make_float2(k0, k0), v2, A0);
+            A1 = __ffma2_rn(make_float2(k1, k1), v2, A1);
             const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
-            h = __ffma2_rn(make_float2(g, g), __fadd2_rn(make_float2(z0, z1), make_float2(-h.x, -h.y)), h);
-            // readout partial of this row: q_t[i]·h_t[i, :]
-            const float qi = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(st + C::ST_Q + (tt * RS + warp) * 2));
-            float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * RS + warp) * V;
-            yb[j0] = qi * h.x;
-            yb[j1] = qi * h.y;
+            {
+                const float z0 = FAST ? tanh_approx(A0.x) : tanh_exp(A0.x);
+                const float z1 = FAST ? tanh_approx(A0.y) : tanh_exp(A0.y);
+                h0 = __ffma2_rn(make_float2(g, g), __fadd2_rn(make_float2(z0, z1), make_float2(-h0.x, -h0.y)), h0);
+                const float z2 = FAST ? tanh_approx(A1.x) : tanh_exp(A1.x);
+                const float z3 = FAST ? tanh_approx(A1.y) : tanh_exp(A1.y);
+                h1 = __ffma2_rn(make_float2(g, g), __fadd2_rn(make_float2(z2, z3), make_float2(-h1.x, -h1.y)), h1);
+            }
+            // readout partials of the two rows: q_t[i]·h_t[i, :]
+            const uint32_t qq = *reinterpret_cast<const uint32_t*>(st + C::ST_Q + (tt * RS + r0) * 2);
+            const float q0 = bf16lo_to_f32(qq), q1 = bf16hi_to_f32(qq);
+            float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * RS + r0) * V;
+            yb[j0] = q0 * h0.x; yb[j1] = q0 * h0.y; yb[V + j0] = q1 * h1.x; yb[V + j1] = q1 * h1.y;
             if (p.ckpt != nullptr && (t + 1) < T && ((t + 1) % p.C) == 0) {
                 float* ck = p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * K * V + (size_t)i * V;
-                ck[j0] = h.x;
-                ck[j1] = h.y;
+                ck[j0] = h0.x; ck[j1] = h0.y; ck[V + j0] = h1.x; ck[V + j1] = h1.y;
             }
             if (tt == C::TC - 1 || t == T - 1) {
                 __syncwarp();
@@ -181,8 +205,7 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             }
         }
         if (ok && p.HT != nullptr) {
-            p.HT[srow + j0] = h.x;
-            p.HT[srow + j1] = h.y;
+            p.HT[srow0 + j0] = h0.x; p.HT[srow0 + j1] = h0.y; p.HT[srow1 + j0] = h1.x; p.HT[srow1 + j1] = h1.y;
         }
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer

@@ -111,9 +111,10 @@ def test_roofline_fraction_counts_one_tanh_per_element():
     assert fast["frac"] == e["frac"] and fast["sfu_ops"]["per_tanh"] == 1
     assert abs(e["tensor"]["achieved_tflops"] - 2 * 64 ** 3 * units / 2e-3 / 1e12) < 1e-6
     assert abs(e["cycles_per_recurrence_step"] - 2e-3 * 1965e6 / w.T) < 1e-6
-    # a CUDA-core (fp32 debug) kernel has no tensor-pipe figure
-    assert "tensor" not in bench.kernel_entry(ms, dict(fwd, flop=0.0), units, w.T, peaks, "measured",
-                                              1965.0, 1965.0)
+    # a CUDA-core kernel reports its product against the derived fp32 FMA peak instead
+    c = bench.kernel_entry(ms, fwd, units, w.T, peaks, "measured", 1965.0, 1965.0, pipe="fma")
+    assert "tensor" not in c and c["fma"]["peak_tflops"] == 148 * 128 * 2 * 1965.0 / 1e6
+    assert bench.kernel_pipe("m2rnn_fwd_rows_kernel") == "fma" and bench.kernel_pipe("m2rnn_bwd_tc_kernel") == "tensor"
 
 
 def test_kernel_digest_covers_the_shared_headers(tmp_path, monkeypatch):
@@ -125,3 +126,26 @@ def test_kernel_digest_covers_the_shared_headers(tmp_path, monkeypatch):
     d1 = bench.kernel_digest(bench.kernel_source("k.cu"))
     (csrc / "ptx.cuh").write_bytes(b"#define A 2\n")
     assert bench.kernel_digest(bench.kernel_source("k.cu")) != d1
+
+
+@pytest.mark.parametrize("B,H,K,V", [(1, 16, 64, 64), (2, 16, 64, 64), (8, 16, 64, 64), (2, 3, 64, 64),
+                                     (1, 16, 128, 64), (1, 4, 16, 64), (2, 3, 64, 32), (4, 32, 128, 128)])
+def test_forward_kernel_rule_matches_the_library(B, H, K, V):
+    """bench.forward_kernel mirrors the library's dispatch; the library shows
+    its choice in the forward workspace: the row kernel keeps K/8 partial
+    readouts per pair, the tensor-core kernel at most K/16."""
+    from non_linear_matrix_persistent_b200 import _lib, build
+    build.build()
+    T = 5
+    w = WORKLOADS["layer410m_fwd"].with_(B=B, H=H, K=K, V=V, T=T)
+    ws = _lib.lib().m2rnn_workspace_size(_lib.Dims(B, H, T, K, V, 0, 16, 0, 0), 0)
+    rows = ws == 256 + (K // 8) * B * H * T * V * 4
+    assert (bench.forward_kernel(w)[0] == "m2rnn_fwd_rows_kernel") == rows
+    assert bench.profile_name(bench.forward_kernel(w)[0], "x") in ("m2rnn_fwd_rows_x.md", "m2rnn_fwd_tc_x.md")
+
+
+def test_backward_kernel_rule():
+    w = WORKLOADS["layer410m_train"]
+    assert bench.backward_kernel(w) == ("m2rnn_bwd_tc_kernel", "bwd_tc.cu")
+    assert bench.backward_kernel(WORKLOADS["layer7b_moe_train"]) == ("m2rnn_bwd_tcg_kernel", "bwd_tcg.cu")
+    assert bench.backward_kernel(w.with_(K=16)) == ("m2rnn_bwd_tcg_kernel", "bwd_tcg.cu")
