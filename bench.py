@@ -449,6 +449,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only the main workload (no forward-only configs)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller cases of the same kernels for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -456,6 +458,8 @@ def main():
     rank, world = parallel.world_from_env()
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.batch > 0:
+        w = w.with_(B=args.batch)
 
     if args.impl == "reference":
         if rank == 0:
