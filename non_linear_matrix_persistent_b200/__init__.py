@@ -7,7 +7,7 @@ import importlib
 
 from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
 
-_API_NAMES = ("forward", "backward", "step", "device_status", "set_wait_limit_ns")
+_API_NAMES = ("forward", "backward", "step", "device_status", "set_wait_limit_ns", "decay_logit_bias")
 
 
 def __getattr__(name):

@@ -6,6 +6,7 @@ device memory and the current stream.  Names follow include/m2rnn.h.
   y, HT, ckpt = forward(k, v, q, f, W, H0=None, ckpt_stride=16, want_ckpt=False)
   grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=16)
   y_t         = step(k_t, v_t, q_t, f_t, W, H)        # one decode step, H updated in place
+  b           = decay_logit_bias(H)                   # per-head gate-logit bias at initialisation
 
 k and q may carry fewer heads than v (G dividing H: grouped k / q, head h
 uses group h // (H // G)); dk and dq then have G heads too.  With
@@ -201,3 +202,23 @@ def device_status(device=None) -> int:
 
 def set_wait_limit_ns(ns: int) -> None:
     _lib.lib().m2rnn_set_wait_limit_ns(int(ns))
+
+
+def decay_logit_bias(H: int, tau_min: float = 2.0, tau_max: float = 256.0) -> torch.Tensor:
+    """Per-head bias of the gate logit at initialisation, shape [H] (fp32, CPU).
+
+    The pages parameterise the forget gate as f_t = ψ(x_t) in [0, 1] and start
+    the heads with different decay rates (gist.science technical summary of
+    "M²RNN", §2.1, forget gate), without giving the form.  This library's
+    reading: ψ ends in the logistic function of a logit a_t = (projection of
+    x_t) + b_h, and at initialisation, where the projection contributes about
+    nothing, head h retains f_h = 1 / (1 + exp(-b_h)) of its state per step.
+    The heads' retention times tau_h = 1 / (1 - f_h) are spaced geometrically
+    from tau_min to tau_max steps, so b_h = log(tau_h - 1).  Pass logits built
+    on it with f_is_logit=True."""
+    if H < 1 or not (1.0 < tau_min <= tau_max):
+        raise ValueError("need H >= 1 and 1 < tau_min <= tau_max")
+    h = torch.arange(H, dtype=torch.float64)
+    frac = h / (H - 1) if H > 1 else torch.zeros(1, dtype=torch.float64)
+    tau = tau_min * (tau_max / tau_min) ** frac
+    return torch.log(tau - 1.0).float()

@@ -584,6 +584,28 @@ def test_gate_logit_backward(mode, K, G, T, C):
     _check_grads("logit_bwd_%s_K%d_G%d_T%d" % (mode, K, G, T), g, gr, GRAD_REL if mode == "bf16" else 1e-4)
 
 
+@pytest.mark.parametrize("K,V", [(64, 64), (128, 128)])
+def test_gate_logits_on_the_decay_bias(K, V):
+    """Gate logits a_t = b_h + noise, with b_h the per-head decay bias of
+    decay_logit_bias (retention times 2 .. 256 steps over the heads), through
+    the forward and the backward against the oracle."""
+    from non_linear_matrix_persistent_b200 import api as a
+    w = Workload("gdb", B=2, H=8, T=45, K=K, V=V, h0_range=0.5, backward=True, gate_logits=True, seed=K + 1)
+    x = make_inputs(w)
+    noise = torch.randn(w.B, w.H, w.T, generator=torch.Generator().manual_seed(3)) * 0.5
+    x["f"] = (a.decay_logit_bias(w.H)[None, :, None] + noise).float().contiguous()
+    xc = _cuda(x)
+    y, HT, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=8, want_ckpt=True,
+                          f_is_logit=True)
+    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=8, f_is_logit=True)
+    torch.cuda.synchronize()
+    assert a.device_status() == 0
+    yr, HTr = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], f_is_logit=True)
+    _check_fwd("decay_bias_fwd_K%d" % K, y, HT, yr, HTr, "bf16")
+    gr = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], f_is_logit=True)
+    _check_grads("decay_bias_bwd_K%d" % K, g, gr, GRAD_REL)
+
+
 def test_gate_logit_decode_steps_match_scan_bitwise():
     w = Workload("gld", B=2, H=2, T=9, K=64, V=64, h0_range=0.5, gate_logits=True, seed=4)
     xc = _cuda(make_inputs(w))
