@@ -21,6 +21,9 @@ resident mma.sync, fp32 debug) and in both backwards, against the fp64
 oracle at the tolerances of the other parity tests.  The last test checks
 the full-size training workload on several heads, pair by pair.
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -36,6 +39,13 @@ DBG_ABS = 1e-4
 GRAD_REL = 1e-2
 NAMES = ("dk", "dv", "dq", "df", "dW", "dH0")
 FWD_VARIANTS = ["tc", "fast", "mma", "fp32"]
+_LOG = os.environ.get("M2RNN_PARITY_LOG")
+
+
+def _log(name, **kw):
+    if _LOG:
+        with open(_LOG, "a") as fh:
+            fh.write(json.dumps(dict(test=name, **kw)) + "\n")
 
 
 def api():
@@ -125,6 +135,7 @@ def test_edge_forward(case, variant, K, V):
     assert api().device_status() == 0
     assert torch.isfinite(y).all() and torch.isfinite(HT).all()
     yr, HTr = oracle.forward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"])
+    _log("edge_fwd_%s_%s_K%d_V%d" % (case, variant, K, V), y_abs=_errs(y, yr)[0], h_abs=_errs(HT, HTr)[0])
     _check_fwd(y, HT, yr, HTr, mode)
     if case == "f1":
         # the state never moves: bit for bit, and the oracle agrees exactly
@@ -158,9 +169,12 @@ def test_edge_backward(case, mode, K, V):
     assert a.device_status() == 0
     gr = oracle.backward(x["k"], x["v"], x["q"], x["f"], x["W"], x["H0"], x["dY"], dHT)
     tol = GRAD_REL if mode == "bf16" else 1e-4
+    rels = {}
     for n in NAMES:
         assert torch.isfinite(g[n]).all(), n
-        _, rel = _errs(g[n], gr[n])
+        _, rels[n] = _errs(g[n], gr[n])
+    _log("edge_bwd_%s_%s_K%d_V%d" % (case, mode, K, V), **rels)
+    for n, rel in rels.items():
         assert rel <= tol, (case, n, rel)
     if case == "f1":
         # dA = (1 - f) G ⊙ (1 - Z²) = 0: no gradient reaches k, v or W, exactly
@@ -209,4 +223,5 @@ def test_train_workload_several_heads_per_pair():
         else:
             rels = [_errs(got[b, i], gr[n][b, i])[1] for b in range(w.B) for i in range(len(heads))]
         worst[n] = max(rels)
+    _log("train_heads_worst_pair", heads=heads, rho=rho[heads].tolist(), **worst)
     assert all(e <= GRAD_REL for e in worst.values()), (heads, rho[heads].tolist(), worst)
