@@ -116,9 +116,12 @@ typedef struct CUstream_st* m2rnn_stream_t;
  * the kernels write before they read it: for the backward, per-(b, h) dW
  * partials and the chunk recompute buffer, plus, when k and q are grouped,
  * the per-head dk and dq (2 · B·H·T·K fp32) summed into the groups' dk and
- * dq at the end; for a tensor-core forward with
- * few (b, h) pairs (B·H·2 <= 148), which splits each pair's K rows over
- * several CTAs, the slices' partial readouts (slices · B·H·T·V fp32). */
+ * dq at the end, and, when V = 128 with K >= 64 (rows split over several
+ * CTAs per pair), the slices' dv and df partials (slices · B·H·T·(V+1) fp32);
+ * for a bf16 forward with few (b, h) pairs, which splits each pair's K rows
+ * over several CTAs (K/8 slices when V = 64 and B·H·K/8 <= 148, else up to 8
+ * slices when B·H·2 <= 148), the slices' partial readouts (slices · B·H·T·V
+ * fp32). */
 size_t m2rnn_workspace_size(const m2rnn_dims* d, int backward);
 
 /* Forward scan.  H0 may be NULL (zero initial state).  HT (final state) and
@@ -143,9 +146,9 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d,
  * it is ckpt[b][h][0], which m2rnn_forward writes from its H0 (zeros for a
  * NULL H0), so the recomputation always starts from the state the forward
  * used and a second copy of H_0 cannot disagree with the checkpoints.  Writes dk, dv, dq, df, dW, dH0 (all
- * required, all fp32).  M2RNN_MODE_BF16_TC supports V = 64, K in
- * {32, 64, 128} and ckpt_stride <= 16 (other shapes return
- * M2RNN_ERR_UNSUPPORTED_SHAPE); M2RNN_MODE_FP32_DEBUG supports every shape. */
+ * required, all fp32).  M2RNN_MODE_BF16_TC supports every K, V in
+ * {16, 32, 64, 128} with ckpt_stride <= 16 (a longer stride returns
+ * M2RNN_ERR_UNSUPPORTED_SHAPE); M2RNN_MODE_FP32_DEBUG supports every stride. */
 m2rnn_status m2rnn_backward(const m2rnn_dims* d,
                             const void* k, const void* v, const void* q,
                             const float* f, const void* W, const float* ckpt,

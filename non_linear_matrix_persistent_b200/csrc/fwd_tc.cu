@@ -9,7 +9,9 @@
 // for all T steps, with the fp32 state in registers.  When there are too few
 // pairs to fill the GPU, a pair's K rows are split over several CTAs (the
 // rows of H are independent given W, v_t and f_t) and the slices' partial
-// readouts are summed by m2rnn_y_reduce_kernel.
+// readouts are summed by m2rnn_y_reduce_kernel; for 64-column states with at
+// most 148 CTAs of 8 rows the row kernel of fwd_rows.cu takes the problem
+// instead (launch_fwd_tc dispatches).
 //
 // Formulation.  The kernel computes the transpose of the transition GEMM,
 //   D = Wᵀ · H_{t-1}ᵀ   (M = V columns of H, N = state rows, contraction V),

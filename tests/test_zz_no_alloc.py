@@ -38,14 +38,17 @@ def _empty_grads(w, dev):
     return {n: torch.full(s, float("nan"), dtype=torch.float32, device=dev) for n, s in shapes.items()}
 
 
-@pytest.mark.parametrize("mode", ["bf16", "fp32"])
-def test_noalloc_backward_matches_workspace_backward(mode):
+@pytest.mark.parametrize("mode,K,V", [("bf16", 64, 64), ("fp32", 64, 64), ("bf16", 128, 128)])
+def test_noalloc_backward_matches_workspace_backward(mode, K, V):
+    """K = V = 128 runs the general-shape tensor-core backward, whose scratch in
+    the array also holds the four row slices' dv and df partials."""
     from non_linear_matrix_persistent_b200 import _lib, api
     C = 8
-    w = Workload("na", B=2, H=3, T=37, K=64, V=64, mode=mode, h0_range=0.5, backward=True, seed=11)
+    w = Workload("na", B=2, H=3, T=37, K=K, V=V, mode=mode, h0_range=0.5, backward=True, seed=11)
     x = make_inputs(w)
     xc = {n: (None if t is None else t.cuda()) for n, t in x.items()}
     dHT = torch.randn(w.B, w.H, w.K, w.V, generator=torch.Generator().manual_seed(2)).cuda()
+    assert _lib.lib().m2rnn_workspace_size(api.dims_of(xc["k"], xc["v"], C), 1) <= (32 << 20)
     _, _, ck = api.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True)
     ref = api.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], dHT, ckpt_stride=C)
     torch.cuda.synchronize()
