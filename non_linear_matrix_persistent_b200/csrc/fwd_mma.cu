@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
             }
         };
         if (p.ckpt != nullptr) store_state(p.ckpt + (size_t)bh * nck * K * V);
+        // next checkpoint step as a running count (no per-step remainder by the run-time stride)
+        int ck_next = p.ckpt != nullptr ? p.C : T + 1, ck_idx = 0;
 
         bool ok = true;
         for (int t = 0; t < T; ++t) {
@@ -203,8 +205,11 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
                 float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES);
                 *reinterpret_cast<float2*>(yb + (warp * C::TC + tt) * V + 8 * g + 2 * tq) = make_float2(pr[0], pr[1]);
             }
-            if (p.ckpt != nullptr && (t + 1) < T && ((t + 1) % p.C) == 0)
-                store_state(p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * K * V);
+            if (t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1} (ck_next lies past T without checkpoints)
+                ck_next += p.C;
+                ++ck_idx;
+                if ((t + 1) < T) store_state(p.ckpt + ((size_t)bh * nck + ck_idx) * K * V);
+            }
             if (tt == C::TC - 1 || t == T - 1) {
                 __syncwarp();
                 if (lane == 0) {

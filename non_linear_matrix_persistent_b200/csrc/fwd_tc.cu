@@ -106,8 +106,14 @@ struct FwdTcCfg {
 };
 
 // FAST: tanh.approx.f32 (one SFU operation, ~2^-11 relative error) instead
-// of the exp-based formula; forward-only inference mode.
-template <int K, int V, bool FAST>
+// of the exp-based formula; forward-only inference mode.  CKPT: the
+// instantiation launched when the call writes checkpoints; it finds the
+// checkpoint steps by a running count (the general path's per-step remainder
+// by the run-time stride cost ~200 cycles per step: 1.71 -> 1.58 ms on the
+// 410M layer).  The other instantiation keeps the general path, whose
+// run-time test never fires without checkpoints; dropping that code altogether
+// measured slower at V = 128 (8.83 -> 9.15 ms) and equal at V = 64.
+template <int K, int V, bool FAST, bool CKPT>
 __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
     using C = FwdTcCfg<K, V>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -186,7 +192,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
         float h[C::RT];
 #pragma unroll
         for (int r = 0; r < C::RT; ++r) h[r] = (p.H0 != nullptr && jv) ? p.H0[sbase + (size_t)(row0 + r) * V + j] : 0.f;
-        if (p.ckpt != nullptr && jv) {
+        if ((CKPT || p.ckpt != nullptr) && jv) {
             float* ck = p.ckpt + (size_t)bh * nck * KF * V + (size_t)koff * V;
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
@@ -197,6 +203,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
         if (lane == 0) mbar_arrive(bready(tile));
 
         const uint32_t tbase = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(tile * C::NT + nsub);
+        int ck_next = p.C, ck_idx = 0;   // CKPT: the next checkpoint step and its index
         bool ok = true;
         for (int t = 0; t < T; ++t) {
             const int c = t / C::TC, tt = t - c * C::TC, s = c % C::S;
@@ -280,7 +287,17 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
                 if (half == 0 && jv)
                     reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES)[(slot * C::TC + tt) * V + j] = yp;
             }
-            if (p.ckpt != nullptr && jv && (t + 1) < T && ((t + 1) % p.C) == 0) {
+            if constexpr (CKPT) {
+                if (t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1}
+                    ck_next += p.C;
+                    ++ck_idx;
+                    if (jv && (t + 1) < T) {
+                        float* ck = p.ckpt + ((size_t)bh * nck + ck_idx) * KF * V + (size_t)koff * V;
+#pragma unroll
+                        for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
+                    }
+                }
+            } else if (p.ckpt != nullptr && jv && (t + 1) < T && ((t + 1) % p.C) == 0) {
                 float* ck = p.ckpt + ((size_t)bh * nck + (t + 1) / p.C) * KF * V + (size_t)koff * V;
 #pragma unroll
                 for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
@@ -412,7 +429,10 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
 template <int K, int V>
 static cudaError_t launch_fwd_tc_kv(const Params& p, cudaStream_t stream) {
     using C = FwdTcCfg<K, V>;
-    auto kern = p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true> : m2rnn_fwd_tc_kernel<K, V, false>;
+    auto kern = p.ckpt != nullptr ? (p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true, true>
+                                                 : m2rnn_fwd_tc_kernel<K, V, false, true>)
+                                  : (p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true, false>
+                                                 : m2rnn_fwd_tc_kernel<K, V, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<p.B * p.H * p.slices, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
