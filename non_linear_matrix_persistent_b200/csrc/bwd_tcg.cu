@@ -11,13 +11,15 @@
 //   df_t  = <G_t, H_{t-1} - Z_t>  dk_t = dA_t v_t      dv_t = dA_tᵀ k_t
 //   dW   += H_{t-1}ᵀ dA_t         G_{t-1} = f_t G_t + dA_t Wᵀ,   dH0 = G_0.
 // As in bwd_tc.cu, each checkpoint chunk of C steps is recomputed from
-// H_{c·C} with the forward's arithmetic (the pages' backward recomputes states
-// rather than storing them, §2.2), its states and Z's go to a workspace
+// H_{c·C} with the forward's epilogue and the state as one bf16 operand (the
+// pages' backward recomputes states rather than storing them, §2.2; the
+// exact fp32 checkpoint every C <= 16 steps bounds that rounding), its states
+// and Z's go to a workspace
 // scratch, and the chunk is then walked in reverse; the recompute of one
 // chunk and the reverse walk of the next run interleaved, each chain with its
 // own accumulators and MMA issuer.  Per step and tile three tcgen05 GEMMs:
-//   recompute      D = Wᵀ · H_{t-1}ᵀ   (M = MX state columns, N = the tile's rows, hi and lo)
-//   G-propagation  D = W · dA_tᵀ       (same shape)
+//   recompute      D = Wᵀ · H_{t-1}ᵀ   (M = MX state columns, N = the tile's rows, bf16 state)
+//   G-propagation  D = W · dA_tᵀ       (N = the tile's rows of dA, hi and lo)
 //   dW             D_W += H_{t-1}ᵀ · dA_t  (M = MX, N = V), accumulated over the sequence
 // with MX = 64 for V <= 64 (rows j >= V of the operands are zero) and 128 for
 // V = 128.  What differs from the V = 64 kernel:
@@ -135,6 +137,13 @@ __device__ __forceinline__ void write_dw_a_operand(uint8_t* Bs, const float (&h)
                                     pack(h[8 * g + 4], h[8 * g + 5]), pack(h[8 * g + 6], h[8 * g + 7]));
         *reinterpret_cast<uint4*>(colbase + ((nloc + 8 * g) >> 3) * 128) = hi;
     }
+}
+
+// Accumulator rows of this thread: the hi half of its RT rows.
+template <class C>
+__device__ __forceinline__ void load_acc_hi(uint32_t taddr, uint32_t (&hi)[C::RT]) {
+    if constexpr (C::MX == 64) tmem_ld_16x32bx2<C::RT, C::RT>(taddr, hi);
+    else tmem_ld_32x32b<C::RT>(taddr, hi);
 }
 
 // Accumulator rows of this thread (hi and lo halves of its RT rows).
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ck_empty);
                 st_vec(Sst, sslot(m, 0), h);
-                if (jv) write_state_operand<C>(Br, h, j, nloc);
+                if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rec(tile));
@@ -432,18 +441,16 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 tc_fence_after();
                 const float vj = bf16_at(str, C::ST_V + u * V * 2);
                 const float g = 1.f - *reinterpret_cast<const float*>(str + C::ST_F + u * 4);
-                uint32_t ahi[C::RT], alo[C::RT];
-                load_acc<C>(tb_rec, ahi, alo);
+                uint32_t ahi[C::RT];
+                load_acc_hi<C>(tb_rec, ahi);
                 float kk[C::RT];
                 lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(str + C::ST_K + u * K * 2) + row0, kk);
                 tc_wait_ld();
                 reg_fence(ahi);
-                reg_fence(alo);
                 float zz[C::RT];
 #pragma unroll
                 for (int r = 0; r < C::RT; ++r) {
-                    float a = __uint_as_float(ahi[r]) + __uint_as_float(alo[r]);
-                    a = fmaf(kk[r], vj, a);
+                    const float a = fmaf(kk[r], vj, __uint_as_float(ahi[r]));
                     zz[r] = tanh_exp(a);
                     h[r] = fmaf(g, zz[r] - h[r], h[r]);
                 }
@@ -451,7 +458,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
                 tc_fence_before();
                 if (u + 1 < lenr) {
-                    if (jv) write_state_operand<C>(Br, h, j, nloc);
+                    if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bready_rec(tile));
@@ -616,7 +623,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
     } else if (warp == C::W_MREC) {
         // ------------------------------------------------------------ MMA issuer: recompute chain
         if (lane == 0) {
-            constexpr uint32_t idesc_f = idesc_bf16_f32(C::MX, C::NT, 0, 1);
+            constexpr uint32_t idesc_f = idesc_bf16_f32(C::MX, C::R, 0, 1);   // the state's hi half only
             const uint32_t w0 = smem_u32(smem + C::OFF_W);
             uint32_t nbr[C::P];
             int issued[C::P];
