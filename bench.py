@@ -39,7 +39,6 @@ from non_linear_matrix_persistent_b200.inputs import make_shard_inputs  # noqa: 
 
 METRIC = "M2RNN layer fwd(+bwd) tokens/s on 1 B200; tensor-pipe % and HBM GB/s via ncu"
 DEFAULT_WORKLOAD = "layer410m_train"
-CKPT_STRIDE = 16
 L2_FLUSH_BYTES = 256 << 20
 NUM_SMS = 148
 SFU_PER_SM_PER_CLK = 16      # special-function (exp / reciprocal / tanh) results per SM per clock
@@ -132,7 +131,7 @@ def per_step_counts(w):
     """Algorithmic work per (b, h, t) of each kernel: tanh count, tensor FLOP
     (one GEMM forward, three backward) and compulsory HBM bytes (bf16 inputs,
     fp32 outputs and gradients, the fp32 checkpoint amortised over C steps)."""
-    K, V, C = w.K, w.V, CKPT_STRIDE
+    K, V, C = w.K, w.V, w.ckpt_stride
     fwd = {"tanh": K * V, "flop": 2.0 * K * V * V,
            "bytes": (2 * K + V) * 2 + 4 + 4 * V + (4.0 * K * V / C if w.backward else 0.0)}
     bwd = {"tanh": K * V, "flop": 3 * 2.0 * K * V * V,
@@ -154,9 +153,10 @@ def forward_kernel(w):
 
 def backward_kernel(w):
     """(kernel name, source file) of the tensor-core backward for workload w:
-    the extended-operand kernel for V = 64 with K >= 32, the general-shape
-    kernel otherwise."""
-    if w.V == 64 and w.K in (32, 64, 128):
+    the extended-operand kernel for V = 64 with K >= 32 and a checkpoint
+    stride that its tensor-memory scratch holds (16 steps at K = 32, 8 at
+    K = 64 and 128), the general-shape kernel otherwise."""
+    if w.V == 64 and w.K in (32, 64, 128) and w.ckpt_stride <= (16 if w.K == 32 else 8):
         return "m2rnn_bwd_tc_kernel", "bwd_tc.cu"
     return "m2rnn_bwd_tcg_kernel", "bwd_tcg.cu"
 
@@ -174,7 +174,7 @@ def launches_per_step(w) -> int:
     reduction for a training workload."""
     from non_linear_matrix_persistent_b200 import _lib
     d = _lib.Dims(w.B, w.H, w.T, w.K, w.V, _lib.MODE_BF16_TC if w.mode == "bf16" else _lib.MODE_FP32_DEBUG,
-                  CKPT_STRIDE, 0, 0)
+                  w.ckpt_stride, 0, 0)
     sliced = _lib.lib().m2rnn_workspace_size(d, 0) > 256
     return 1 + (1 if sliced else 0) + (2 if w.backward else 0)
 
@@ -352,7 +352,7 @@ def time_training_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_m
     from non_linear_matrix_persistent_b200 import api
     w = WORKLOADS[name]
     x = make_inputs(w, device=str(dev))
-    B, H, T, K, V, C = w.B, w.H, w.T, w.K, w.V, CKPT_STRIDE
+    B, H, T, K, V, C = w.B, w.H, w.T, w.K, w.V, w.ckpt_stride
     out = {"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev),
            "ckpt": torch.empty(B, H, (T + C - 1) // C, K, V, device=dev)}
     gout = {}
@@ -396,7 +396,7 @@ def time_training_config(name, steps, warmup, dev, flush, peaks, peak_kind, sm_m
 
 def bench_config(w, world):
     """The workload description both arms print (same keys, same values)."""
-    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "K": w.K, "V": w.V, "ckpt_stride": CKPT_STRIDE,
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "K": w.K, "V": w.V, "ckpt_stride": w.ckpt_stride,
             "global_batch": w.B * world, "seq_len": w.T, "parallelism": "dp%d" % world,
             "l2": "flushed between timed steps (256 MB write)"}
 
@@ -474,7 +474,7 @@ def main():
     from non_linear_matrix_persistent_b200 import api
     x_host = make_shard_inputs(w, rank)
     x = {n: (None if t is None else t.to(dev)) for n, t in x_host.items()}
-    C = CKPT_STRIDE
+    C = w.ckpt_stride
     B, H, T, K, V = w.B, w.H, w.T, w.K, w.V
     outs = {"y": torch.empty(B, H, T, V, device=dev), "HT": torch.empty(B, H, K, V, device=dev),
             "ckpt": torch.empty(B, H, (T + C - 1) // C, K, V, device=dev)}

@@ -114,7 +114,9 @@ typedef struct CUstream_st* m2rnn_stream_t;
  * Returns 0 for invalid dims.  The first 256 bytes hold the device status
  * word: zero them once after allocating the workspace.  The rest is scratch
  * the kernels write before they read it: for the backward, per-(b, h) dW
- * partials and the chunk recompute buffer, plus, when k and q are grouped,
+ * partials and, except for V = 64 with a stride of at most 8 (16 for
+ * K = 32), whose chunk stays on chip, the chunk recompute buffer, plus,
+ * when k and q are grouped,
  * the per-head dk and dq (2 · B·H·T·K fp32) summed into the groups' dk and
  * dq at the end, and, when V = 128 with K >= 64 (rows split over several
  * CTAs per pair), the slices' dv and df partials (slices · B·H·T·(V+1) fp32);
@@ -148,7 +150,9 @@ m2rnn_status m2rnn_forward(const m2rnn_dims* d,
  * used and a second copy of H_0 cannot disagree with the checkpoints.  Writes dk, dv, dq, df, dW, dH0 (all
  * required, all fp32).  M2RNN_MODE_BF16_TC supports every K, V in
  * {16, 32, 64, 128} with ckpt_stride <= 16 (a longer stride returns
- * M2RNN_ERR_UNSUPPORTED_SHAPE); M2RNN_MODE_FP32_DEBUG supports every stride. */
+ * M2RNN_ERR_UNSUPPORTED_SHAPE); for V = 64 and K >= 32 a stride of at most 8
+ * (16 for K = 32) takes the faster kernel, which keeps the recomputed chunk
+ * on chip.  M2RNN_MODE_FP32_DEBUG supports every stride. */
 m2rnn_status m2rnn_backward(const m2rnn_dims* d,
                             const void* k, const void* v, const void* q,
                             const float* f, const void* W, const float* ckpt,

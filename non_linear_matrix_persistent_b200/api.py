@@ -3,8 +3,8 @@
 Every step of the recurrence runs in the CUDA library; torch only provides
 device memory and the current stream.  Names follow include/m2rnn.h.
 
-  y, HT, ckpt = forward(k, v, q, f, W, H0=None, ckpt_stride=16, want_ckpt=False)
-  grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=16)
+  y, HT, ckpt = forward(k, v, q, f, W, H0=None, ckpt_stride=8, want_ckpt=False)
+  grads       = backward(k, v, q, f, W, ckpt, dy, dHT=None, ckpt_stride=8)
   y_t         = step(k_t, v_t, q_t, f_t, W, H)        # one decode step, H updated in place
   b           = decay_logit_bias(H)                   # per-head gate-logit bias at initialisation
 
@@ -17,6 +17,10 @@ bf16 k/v/q/W select the tensor-core mode (M2RNN_MODE_BF16_TC); fp32 select
 the fp32 debug mode; forward(..., fast_tanh=True) and forward(...,
 mma_sync=True) select the forward-only alternatives.  Tensors must be
 contiguous CUDA tensors with the head-first layouts of the header.
+
+The default checkpoint stride, 8, is the longest chunk that the V = 64
+tensor-core backward keeps in tensor memory for K = 64 and 128 (16 for
+K = 32); longer strides (up to 16) run the general-shape backward.
 """
 from __future__ import annotations
 
@@ -59,7 +63,7 @@ def _check(name, t, shape, dtype, device):
         raise ValueError("%s must be contiguous" % name)
 
 
-def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 16, f_is_logit: bool = False) -> Dims:
+def dims_of(k: torch.Tensor, v: torch.Tensor, ckpt_stride: int = 8, f_is_logit: bool = False) -> Dims:
     """Dims of a call: H from v, the k / q head groups G from k."""
     B, G, T, K = k.shape
     H = v.shape[1]
@@ -95,7 +99,7 @@ def num_checkpoints(T: int, ckpt_stride: int) -> int:
     return (T + ckpt_stride - 1) // ckpt_stride
 
 
-def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 16, want_ckpt: bool = False,
+def forward(k, v, q, f, W, H0=None, *, ckpt_stride: int = 8, want_ckpt: bool = False,
             want_HT: bool = True, out: Optional[dict] = None, fast_tanh: bool = False,
             mma_sync: bool = False, f_is_logit: bool = False):
     """Runs the forward scan.  Returns (y, HT or None, ckpt or None).
@@ -158,7 +162,7 @@ def step(k, v, q, f, W, H, *, y: Optional[torch.Tensor] = None, f_is_logit: bool
     return y
 
 
-def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 16, out: Optional[dict] = None,
+def backward(k, v, q, f, W, ckpt, dy, dHT=None, *, ckpt_stride: int = 8, out: Optional[dict] = None,
              f_is_logit: bool = False):
     """BPTT from the forward's checkpoints.  Returns dict dk, dv, dq, df, dW, dH0 (fp32)."""
     dev = k.device

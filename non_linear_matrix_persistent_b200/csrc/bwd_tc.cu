@@ -14,13 +14,15 @@
 // H_{c·C} with the forward kernel's epilogue, but with the state entering the
 // recompute product as one bf16 operand (round to nearest) rather than the
 // forward's compensated hi + lo pair: each chunk restarts from an exact fp32
-// checkpoint, so the rounding cannot accumulate beyond C <= 16 steps, and on
-// three full heads of the 410M training workload every (b, h) pair's
-// gradients stayed as close to the fp64 oracle as with the pair (worst dW
-// 6.0e-3 against 6.3e-3; dq 1.9e-3 against 8.8e-5) while the backward took
-// 3.70 instead of 3.81 ms.  H_{t-1} and Z_t of the chunk go to a workspace
-// scratch (read back only by the thread that wrote them), then the chunk is
-// walked in reverse.
+// checkpoint, so the rounding cannot accumulate beyond C steps, and on three
+// full heads of the 410M training workload every (b, h) pair's gradients
+// stayed as close to the fp64 oracle as with the pair (worst dW 6.0e-3
+// against 6.3e-3; dq 1.9e-3 against 8.8e-5).  The chunk's Z_t stay in tensor
+// memory (fp32, read back only by the thread that wrote them) and its states
+// in a shared-memory ring of bf16 MMA operands, then the chunk is walked in
+// reverse.  (With the chunk in a global-memory scratch instead, its round
+// trip through L2 cost 22% of the backward: 3.75 ms against 2.93 ms with the
+// scratch traffic removed, at C = 16.)
 //
 // Layout: one CTA per (b, h) and slice of at most 64 state rows (rows of H
 // evolve independently given W, v_t and f_t), the slice's rows split into
@@ -37,11 +39,13 @@
 // otherwise take cross-lane shuffles:
 //   recompute:      Σ_l dy_{t-1}[l] H_{t-1}[i, l] = dq_{t-1}[i]
 //   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
-// Software pipelining: the recompute of one chunk and the reverse walk of
-// the chunk after it (in time) are independent chains, so the epilogue
-// interleaves them step for step, each with its own TMEM accumulators and
-// MMA issuer warp, sharing one scratch buffer; each chain's MMA round trip
-// overlaps the other chain's epilogue work.
+// The G-propagation MMA takes dA as a compensated pair (hi, then lo rows of
+// its operand) and sums both halves in one accumulator, two MMA groups of
+// N = R.  Software pipelining: the recompute of one chunk and the reverse
+// walk of the chunk after it (in time) are independent chains, so the
+// epilogue interleaves them step for step, each with its own TMEM
+// accumulators and MMA issuer warp, sharing the scratch; each chain's MMA
+// round trip overlaps the other chain's epilogue work.
 // dv, df are thread-local plus shuffles; their per-warp partials are summed
 // in a fixed order by a storer warp (with two slices, added into a zeroed
 // output, which is order-independent for two addends), and the dW partials
@@ -55,8 +59,9 @@
 // dL/df_t · f_t (1 - f_t) (gate_grad).  The epilogue stays scalar: packed
 // fp32 pairs, which help the forward, measured slower here.
 //
-// Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 16; the other
-// shapes run the general-shape kernel of bwd_tcg.cu.
+// Supported: V = 64, K in {32, 64, 128}, checkpoint stride C <= 8 (C <= 16
+// for K = 32), the chunk that the tensor-memory scratch holds; the other
+// shapes and strides run the general-shape kernel of bwd_tcg.cu.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -77,16 +82,21 @@ struct BwdTcCfg {
     static constexpr int MX = 128;            // M of the recompute and G-propagation MMAs
     static constexpr int XLANE = 16;          // TMEM lane (and Ã row) of the extra output
     static constexpr int R = K / P;           // rows per tile
-    static constexpr int NT = 2 * R;          // MMA N per tile (hi rows, then lo rows)
+    static constexpr int NT = 2 * R;          // G-propagation MMA N per tile (dA hi rows, then lo rows)
     // two warps per TMEM lane quarter and tile (each owning half of the tile's
     // rows) when the tile is large enough: the epilogue is issue-bound, and
     // more warps with fewer rows each raise the issue rate
     static constexpr int SUBS = (R / 4 >= 4) ? 2 : 1;
     static constexpr int WPT = 4 * SUBS;      // epilogue warps per tile
     static constexpr int RT = R / (2 * SUBS); // rows per epilogue thread
-    static constexpr int CMAX = 16;           // max steps per checkpoint chunk
     static constexpr int NWE = P * WPT;       // epilogue warps
-    static constexpr int NSLOT = P * SUBS;    // dv partials per (t, j)
+    static constexpr int NSLOT = P * SUBS;    // dv partials per (t, j); also the epilogue warps per lane quarter
+    // Recompute scratch in tensor memory: per step, one 32-bit column per
+    // state element (1 - Z² and Z - H_{t-1} as an fp16 pair), a lane quarter's
+    // NSLOT warps with RT columns each; SCR_COLS columns hold CMAX steps.
+    static constexpr int SCR_COL = 256, SCR_COLS = 256;
+    static constexpr int SCR_STEP = NSLOT * RT;
+    static constexpr int CMAX = SCR_COLS / SCR_STEP < 16 ? SCR_COLS / SCR_STEP : 16;   // max steps per chunk
     // service warps; the two readers of TMEM lane XLANE sit in lane quarter 0
     static constexpr int W_XD = NWE, W_MREV = NWE + 1, W_MREC = NWE + 2, W_STORE = NWE + 3, W_XQ = NWE + 4,
                          W_PROD = NWE + 5;
@@ -94,7 +104,9 @@ struct BwdTcCfg {
     static constexpr int NSTAGE = 3;          // input chunks: recompute of i, reverse of i-1, prefetch of i+1
 
     static constexpr int AX_BYTES = MX * V * 2;            // one extended A operand
-    static constexpr int B_BYTES = NT * V * 2;
+    static constexpr int B_BYTES = NT * V * 2;             // one tile's dA operand (hi + lo)
+    static constexpr int BR_BYTES = R * V * 2;             // one tile's state operand (bf16, R rows)
+    static constexpr int NBR = CMAX + 2;                   // state-operand ring slots (see the epilogue)
     static constexpr int ST_K = 0;
     static constexpr int ST_Q = CMAX * KF * 2;   // k and q rows hold all KF values
     static constexpr int ST_V = 2 * CMAX * KF * 2;
@@ -107,10 +119,9 @@ struct BwdTcCfg {
 
     static constexpr int OFF_AF = 0;                       // Ã_f per tile (K-major)
     static constexpr int OFF_AG = OFF_AF + P * AX_BYTES;   // Ã_g per tile (MN-major)
-    static constexpr int OFF_BR = OFF_AG + P * AX_BYTES;   // recompute state operands
-    static constexpr int OFF_BS = OFF_BR + P * B_BYTES;    // H_{t-1} operands of the dW MMA
-    static constexpr int OFF_BD = OFF_BS + P * B_BYTES;    // dA operands
-    static constexpr int OFF_RING = OFF_BD + P * B_BYTES;
+    static constexpr int OFF_BD = OFF_AG + P * AX_BYTES;   // dA operands
+    static constexpr int OFF_BR = OFF_BD + P * B_BYTES;    // state operands, [NBR][P]
+    static constexpr int OFF_RING = OFF_BR + NBR * P * BR_BYTES;
     static constexpr int OFF_CK = OFF_RING + NSTAGE * STAGE_BYTES;   // the next checkpoint (fp32 [K][V])
     static constexpr int OFF_PART = OFF_CK + K * V * 4;
     // dv / df partials: double-buffered when shared memory allows, so the
@@ -121,18 +132,19 @@ struct BwdTcCfg {
     // partial buffer, ck_full/ck_empty
     static constexpr int NBAR = 2 * NSTAGE + 4 * P + 2 * NPART + 2;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
-    static constexpr int REV_COL = 0;                      // G-propagation accumulators, NT columns per tile
-    static constexpr int REC_COL = P * NT;                 // recompute accumulators
-    static constexpr int DW_COL = 2 * P * NT;              // dW accumulator (V columns)
-    static constexpr int TMEM_COLS = (DW_COL + V <= 128) ? 128 : (DW_COL + V <= 256) ? 256 : 512;
+    static constexpr int REV_COL = 0;                      // G-propagation accumulators, R columns per tile
+    static constexpr int REC_COL = P * R;                  // recompute accumulators, R columns per tile
+    static constexpr int DW_COL = REC_COL + P * R;         // dW accumulator (V columns)
+    static constexpr int TMEM_COLS = 512;
 
     static_assert(K == 32 || K == 64, "slice rows");
     static_assert(R % 16 == 0, "dW MMA needs 16-row k-steps");
     static_assert(NT % 16 == 0 && NT <= 256, "N of an M = 128 MMA");
-    static_assert(RT % 4 == 0 && NWE * 32 * RT == K * V, "row split");
+    static_assert(RT % 4 == 0 && RT <= 8 && NWE * 32 * RT == K * V, "row split");
     static_assert(NTHREADS <= 1024, "block size");
     static_assert(W_XD % 4 == 0 && W_XQ % 4 == 0, "lane-quarter 0 readers");
-    static_assert(DW_COL + V <= 512, "TMEM columns");
+    static_assert(DW_COL + V <= SCR_COL && SCR_COL + SCR_COLS <= TMEM_COLS, "TMEM columns");
+    static_assert(CMAX >= 8, "checkpoint stride");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
 
@@ -147,34 +159,24 @@ __device__ __forceinline__ int ag_off(int m, int k) {
     return (k >> 3) * (128 * 16) + (m >> 3) * 128 + (k & 7) * 16 + (m & 7) * 2;
 }
 
-// Stores the extra output row (TMEM lane XLANE) of one tile, hi + lo parts
-// of its R columns summed, to dst[0 .. R).  Warp-collective over lane quarter
-// 0; thread XLANE stores, and only when `store` is set.
-// LO: the MMA's B operand had a lo half (R more columns of D to add).
-template <class C, bool LO>
+// Stores the extra output row (TMEM lane XLANE) of one tile, its R columns,
+// to dst[0 .. R).  Warp-collective over lane quarter 0; thread XLANE stores,
+// and only when `store` is set.
+template <class C>
 __device__ __forceinline__ void store_xrow(uint32_t tcol, float* dst, bool store) {
     constexpr int CHK = C::R < 16 ? C::R : 16;
 #pragma unroll
     for (int c0 = 0; c0 < C::R; c0 += CHK) {
-        uint32_t hi[CHK], lo[CHK];
-        tmem_ld_32x32b<CHK>(tcol + c0, hi);
-        if constexpr (LO) {
-            tmem_ld_32x32b<CHK>(tcol + C::R + c0, lo);
-        } else {
-#pragma unroll
-            for (int e = 0; e < CHK; ++e) lo[e] = 0u;
-        }
+        uint32_t x[CHK];
+        tmem_ld_32x32b<CHK>(tcol + c0, x);
         tc_wait_ld();
-        reg_fence(hi);
-        reg_fence(lo);
+        reg_fence(x);
         if (store) {
             float4* d = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
             for (int g = 0; g < CHK / 4; ++g)
-                d[g] = make_float4(__uint_as_float(hi[4 * g]) + __uint_as_float(lo[4 * g]),
-                                   __uint_as_float(hi[4 * g + 1]) + __uint_as_float(lo[4 * g + 1]),
-                                   __uint_as_float(hi[4 * g + 2]) + __uint_as_float(lo[4 * g + 2]),
-                                   __uint_as_float(hi[4 * g + 3]) + __uint_as_float(lo[4 * g + 3]));
+                d[g] = make_float4(__uint_as_float(x[4 * g]), __uint_as_float(x[4 * g + 1]),
+                                   __uint_as_float(x[4 * g + 2]), __uint_as_float(x[4 * g + 3]));
         }
     }
 }
@@ -266,70 +268,49 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         const int nsub = sub * (C::R / C::SUBS);   // first tile row of this warp
         const int nloc = nsub + half * C::RT;      // first tile row of this thread
         const int row0 = tile * C::R + nloc;
-        const int slot = tile * C::SUBS + sub;
+        const int slot = tile * C::SUBS + sub;     // this warp's index within its lane quarter
         const bool xwriter = sub == 0 && half == 0;            // writes element j of the extra A rows
         const size_t sbase = ((size_t)bh * KF + koff) * V;   // this slice's rows of dH_T / dH0
-        uint8_t* Br = smem + C::OFF_BR + tile * C::B_BYTES;
-        uint8_t* Bs = smem + C::OFF_BS + tile * C::B_BYTES;
         uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
         uint16_t* xf = reinterpret_cast<uint16_t*>(smem + C::OFF_AF + tile * C::AX_BYTES + af_off(C::XLANE, j));
         uint16_t* xg = reinterpret_cast<uint16_t*>(smem + C::OFF_AG + tile * C::AX_BYTES + ag_off(C::XLANE, j));
         const uint32_t lanes = (uint32_t)(qd * 32) << 16;
-        const uint32_t tb_rev = tmem + (uint32_t)(C::REV_COL + tile * C::NT + nsub) + lanes;
-        const uint32_t tb_rec = tmem + (uint32_t)(C::REC_COL + tile * C::NT + nsub) + lanes;
-        // Scratch per CTA: C slots of states (H_{c0+u}, the state before step
-        // c0+u) and C slots of Z_{c0+u}.  One buffer serves both chains: the
-        // chunk recomputed in phase i stores step u in slot u for even i and in
-        // slot C-1-u for odd i, so in phase i+1 the recompute writes exactly
+        const uint32_t tb_rev = tmem + (uint32_t)(C::REV_COL + tile * C::R + nsub) + lanes;
+        const uint32_t tb_rec = tmem + (uint32_t)(C::REC_COL + tile * C::R + nsub) + lanes;
+        // Recompute scratch, in tensor memory: for step c0+u of a chunk, thread
+        // (lane l of warp w) keeps Z_{c0+u} of its RT elements, fp32, in lane
+        // 32·(w mod 4) + l, columns SCR_COL + x·SCR_STEP + slot·RT + r, where x
+        // is the step's scratch slot.  The reverse step's other operand,
+        // H_{t-1}, comes from the state-operand ring below (bf16, rounded to
+        // nearest): it enters only df = <G, H_{t-1} - Z> there, while
+        // dA = (1-f) G (1 - Z²), which the carry G propagates, keeps the fp32 Z
+        // (an fp16 (1 - Z², Z - H_{t-1}) pair in one column was measured: its
+        // rounding, carried back through G, took the worst (b, h) pair's
+        // gradients from 6e-3 to 9e-3 of the oracle's).  One set of CMAX slots serves both chains: the
+        // chunk recomputed in phase i stores step u in slot u for even i and
+        // in slot C-1-u for odd i, so in phase i+1 the recompute writes exactly
         // the slots the reverse walk (which reads its chunk from step len-1
-        // down, one step ahead) has already read.  Slot-major across CTAs:
-        // slot x of CTA b is the K·V block x·nCTA + b, so that the CTAs, which
-        // all touch the same slot at about the same time, hit one contiguous
-        // range instead of addresses a power of two apart (measured 2.5%
-        // faster).  Within a block, thread t holds its RT values at t·RT
-        // (each warp one contiguous run); only the thread that wrote a value
-        // reads it back.
-        const size_t nct = gridDim.x;
-        float* const Sst = p.scratch + (size_t)blockIdx.x * K * V;
-        float* const Sz = Sst + (size_t)CS * nct * K * V;
+        // down, one step ahead) has already read.  Only the thread that wrote
+        // a value reads it back.
+        const uint32_t scr = tmem + lanes + (uint32_t)(C::SCR_COL + slot * C::RT);
         auto sslot = [&](int i, int u) { return (i & 1) ? CS - 1 - u : u; };
-        const size_t tslot = (size_t)threadIdx.x * C::RT;
-        // The scratch (2·C·K·V·4 bytes per CTA, ~64 MB for 128 CTAs at C = 16,
-        // K = V = 64) is stored with L2 evict_last priority, so its round trip
-        // stays in L2 instead of being written back to HBM and read again.
-        const uint64_t pol_keep = l2_policy_evict_last();
-        // 32-byte accesses when the workspace allows (it is 32-byte aligned in
-        // practice; the ABI promises 16): each thread's RT values are RT·4 bytes
-        // at a multiple of RT·4
-        const bool v8 = C::RT % 8 == 0 && (reinterpret_cast<uintptr_t>(Sst) & 31) == 0;
-        auto st_vec = [&](float* base, int u, const float (&v)[C::RT]) {
-            float* d = base + (size_t)u * nct * K * V + tslot;
-            if (v8) {
-#pragma unroll
-                for (int g = 0; g < C::RT / 8; ++g) st_global_v8_hint(d + 8 * g, v + 8 * g, pol_keep);
-            } else {
-#pragma unroll
-                for (int g = 0; g < C::RT / 4; ++g)
-                    st_global_v4_hint(d + 4 * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3], pol_keep);
-            }
-        };
-        auto ld_vec = [&](const float* base, int u, float (&v)[C::RT]) {
-            const float* src = base + (size_t)u * nct * K * V + tslot;
-            if (v8) {
-#pragma unroll
-                for (int g = 0; g < C::RT / 8; ++g) ld_global_v8(src + 8 * g, v + 8 * g);
-            } else {
-                const float4* s4 = reinterpret_cast<const float4*>(src);
-#pragma unroll
-                for (int g = 0; g < C::RT / 4; ++g) {
-                    const float4 x = s4[g];
-                    v[4 * g] = x.x; v[4 * g + 1] = x.y; v[4 * g + 2] = x.z; v[4 * g + 3] = x.w;
-                }
-            }
-        };
+        auto scr_at = [&](int x) { return scr + (uint32_t)(x * C::SCR_STEP); };
+        // State operands H_{c0+u} (bf16, round to nearest) in a ring of CS + 2
+        // slots per tile: the recompute MMA of step c0+u reads slot x(u), and
+        // so does, one phase later, the dW MMA of the same step.  The mirror
+        // order (slot u for even phases, CS+1-u for odd ones) with two spare
+        // slots keeps every write of a phase's recompute off the slots whose
+        // dW MMA is still to be issued or still running (the reverse walk reads
+        // its chunk from the top down while the recompute writes from the
+        // bottom up; the dW MMA of reverse step s may run until reverse step
+        // s+1 starts, one step after the epilogue's own reads).
+        auto bslot = [&](int i, int u) { return (i & 1) ? CS + 1 - u : u; };
+        auto Br = [&](int x) { return smem + C::OFF_BR + (x * C::P + tile) * C::BR_BYTES; };
         auto stage = [&](int i) { return smem + C::OFF_RING + (i % C::NSTAGE) * C::STAGE_BYTES; };
 
-        float G[C::RT], h[C::RT], zc[C::RT], hpc[C::RT];
+        float G[C::RT], h[C::RT];
+        uint32_t sz[C::RT];   // Z of the next reverse step (fp32 bits)
+        float hp[C::RT];      // its H_{t-1} (bf16 values), from the ring slot its dW MMA reads
 #pragma unroll
         for (int r = 0; r < C::RT; ++r) G[r] = p.dHT != nullptr ? p.dHT[sbase + (size_t)(row0 + r) * V + j] : 0.f;
         float fprev = 0.f;
@@ -361,9 +342,10 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                                     mbar_wait_bounded(pempty(pb), ((i / C::NPART) - 1) & 1, abort_flag, p));
                     if (!ok) break;
                 }
-                // before the recompute below stores its first state (same slot)
-                ld_vec(Sz, sslot(m - 1, lenv - 1), zc);
-                ld_vec(Sst, sslot(m - 1, lenv - 1), hpc);
+                // before the recompute below stores its first step (same slot)
+                tc_wait_st();
+                tmem_ld_32x32b<C::RT>(scr_at(sslot(m - 1, lenv - 1)), sz);
+                read_state_operand_hi<C, C::R>(Br(bslot(m - 1, lenv - 1)), j, nloc, hp);
             }
             if (has_rec) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(m % C::NSTAGE), (m / C::NSTAGE) & 1, abort_flag, p));
@@ -375,8 +357,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 for (int r = 0; r < C::RT; ++r) h[r] = ck[(row0 + r) * V + j];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ck_empty);
-                st_vec(Sst, sslot(m, 0), h);
-                write_state_operand_hi<C>(Br, h, j, nloc);
+                write_state_operand_hi<C, C::R>(Br(bslot(m, 0)), h, j, nloc);
                 if (xwriter) *xf = c0r > 0 ? dyr(-1)[j] : (uint16_t)0;
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -386,20 +367,28 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
             auto rev_step = [&](int s) -> bool {
                 // ---------------------------------------- reverse step t = c0v + u
                 const int u = lenv - 1 - s;
+                // this step's scratch terms, before the wait for the G-propagation
+                // result, so that they stay off the chain from that result to dA_t
+                tc_wait_ld();   // the Z prefetched by the previous reverse step (or the phase start)
+                reg_fence(sz);
+                float sq[C::RT], dz[C::RT];   // 1 - Z_t², H_{t-1} - Z_t
+#pragma unroll
+                for (int r = 0; r < C::RT; ++r) {
+                    const float z = __uint_as_float(sz[r]);
+                    sq[r] = fmaf(-z, z, 1.f);
+                    dz[r] = hp[r] - z;
+                }
                 if (s > 0) {   // fold in dA_{t+1} Wᵀ from the previous reverse step
                     ok = __all_sync(0xffffffffu, mbar_wait_bounded(accfull_rev(tile), nrev & 1, abort_flag, p));
                     if (!ok) return false;
                     ++nrev;
                     tc_fence_after();
-                    uint32_t dhi[C::RT], dlo[C::RT];
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
+                    uint32_t dg[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dg);
                     tc_wait_ld();
-                    reg_fence(dhi);
-                    reg_fence(dlo);
+                    reg_fence(dg);
 #pragma unroll
-                    for (int r = 0; r < C::RT; ++r)
-                        G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                    for (int r = 0; r < C::RT; ++r) G[r] = fmaf(fprev, G[r], __uint_as_float(dg[r]));
                     tc_fence_before();
                 }
                 const float dyj = bf16lo_to_f32(*reinterpret_cast<const uint16_t*>(stv + C::ST_DY + (u + 1) * V * 2 + j * 2));
@@ -412,21 +401,20 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 float dfp = 0.f, dvp = 0.f;
 #pragma unroll
                 for (int r = 0; r < C::RT; ++r) {
-                    const float z = zc[r];
                     G[r] = fmaf(qq[r], dyj, G[r]);
-                    dA[r] = (1.f - ft) * G[r] * fmaf(-z, z, 1.f);
-                    dfp = fmaf(G[r], hpc[r] - z, dfp);
+                    dA[r] = (1.f - ft) * G[r] * sq[r];
+                    dfp = fmaf(G[r], dz[r], dfp);
                     dvp = fmaf(dA[r], kk[r], dvp);
                 }
                 write_state_operand<C, true>(Bd, dA, j, nloc);
-                write_state_operand_hi<C>(Bs, hpc, j, nloc);   // the dW MMA reads the hi half only
                 if (xwriter) *xg = vbits;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rev(tile));
-                if (u > 0) {
-                    ld_vec(Sz, sslot(m - 1, u - 1), zc);
-                    ld_vec(Sst, sslot(m - 1, u - 1), hpc);
+                if (u > 0) {   // the next reverse step's operands, ahead of the recompute step that reuses the slot
+                    tc_wait_st();
+                    tmem_ld_32x32b<C::RT>(scr_at(sslot(m - 1, u - 1)), sz);
+                    read_state_operand_hi<C, C::R>(Br(bslot(m - 1, u - 1)), j, nloc, hp);
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
@@ -436,8 +424,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 fprev = ft;
                 return true;
             };
-            // one recompute step (after the reverse step of the same s, which may
-            // still have to read the scratch slot this one writes)
+            // one recompute step (after the reverse step of the same s, which has
+            // already loaded the scratch slot this one writes)
             auto rec_step = [&](int s) -> bool {
                 // ---------------------------------------- recompute step c0r + u
                 const int u = s;
@@ -453,21 +441,21 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                     tmem_ld_16x32bx2<C::RT, C::RT>(tb_rec, ahi);
                     float kk[C::RT];
                     lds_bf16<C::RT>(reinterpret_cast<const uint16_t*>(str + C::ST_K + u * KF * 2) + koff + row0, kk);
-                    tc_wait_ld();
+                    tc_wait_ld();   // also completes the reverse step's scratch load of this slot
                     reg_fence(ahi);
-                    float zz[C::RT];
+                    uint32_t st[C::RT];
 #pragma unroll
                     for (int r = 0; r < C::RT; ++r) {
                         const float a = fmaf(kk[r], vj, __uint_as_float(ahi[r]));
-                        zz[r] = tanh_exp(a);
-                        h[r] = fmaf(g, zz[r] - h[r], h[r]);
+                        const float z = tanh_exp(a);
+                        st[r] = __float_as_uint(z);
+                        h[r] = fmaf(g, z - h[r], h[r]);
                     }
-                    st_vec(Sz, sslot(m, u), zz);
-                    if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
+                    tmem_st_32x32b<C::RT>(scr_at(sslot(m, u)), st);
                 }
                 tc_fence_before();
                 if (u + 1 < nmr) {
-                    write_state_operand_hi<C>(Br, h, j, nloc);
+                    write_state_operand_hi<C, C::R>(Br(bslot(m, u + 1)), h, j, nloc);
                     if (xwriter) *xf = dyr(u)[j];
                     fence_proxy_async_smem();
                     __syncwarp();
@@ -490,15 +478,12 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 ++nrev;
                 tc_fence_after();
                 {
-                    uint32_t dhi[C::RT], dlo[C::RT];
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dhi);
-                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev + C::R, dlo);
+                    uint32_t dg[C::RT];
+                    tmem_ld_16x32bx2<C::RT, C::RT>(tb_rev, dg);
                     tc_wait_ld();
-                    reg_fence(dhi);
-                    reg_fence(dlo);
+                    reg_fence(dg);
 #pragma unroll
-                    for (int r = 0; r < C::RT; ++r)
-                        G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
+                    for (int r = 0; r < C::RT; ++r) G[r] = fmaf(fprev, G[r], __uint_as_float(dg[r]));
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -508,6 +493,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 }
             }
         }
+        tc_wait_st();   // no scratch store may still be in flight when the columns are freed
         if (ok) {
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) p.dH0[sbase + (size_t)(row0 + r) * V + j] = G[r];
@@ -537,12 +523,11 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                                                                     abort_flag, p));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t tcol = tmem + (uint32_t)((xd ? C::REV_COL : C::REC_COL) + tile * C::NT);
+                    const uint32_t tcol = tmem + (uint32_t)((xd ? C::REV_COL : C::REC_COL) + tile * C::R);
                     float* dst = out + ((size_t)bh * T + max(t, 0)) * KF + koff + tile * C::R;
-                    if (xd)
-                        store_xrow<C, true>(tcol, dst, lane == C::XLANE && t >= 0);
-                    else   // the recompute's state operand has no lo half
-                        store_xrow<C, false>(tcol, dst, lane == C::XLANE && t >= 0);
+                    // (both accumulators are R columns: the G-propagation sums dA's hi and
+                    // lo halves in the MMA, and the recompute's state operand has no lo half)
+                    store_xrow<C>(tcol, dst, lane == C::XLANE && t >= 0);
                     tc_fence_before();
                     __syncwarp();
                     if (!last && lane == 0) mbar_arrive(xd ? bready_rev(tile) : bready_rec(tile));
@@ -603,7 +588,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
     } else if (warp == C::W_MREV) {
         // ------------------------------------------------------------ MMA issuer: reverse chain
         if (lane == 0) {
-            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::NT, 1, 1);
+            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::R, 1, 1);   // dA hi, then dA lo, one accumulator
             constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
             uint32_t nbr[C::P];
             int issued[C::P];
@@ -625,17 +610,26 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                         ++nbr[tile];
                         tc_fence_after();
                         const uint32_t ag = smem_u32(smem + C::OFF_AG + tile * C::AX_BYTES);
-                        const uint32_t bs = smem_u32(smem + C::OFF_BS + tile * C::B_BYTES);
+                        // H_{t-1} of reverse step u (chunk-local step len-1-u) in the
+                        // state-operand ring, in the slot order of the epilogue
+                        const int us = len - 1 - u;
+                        const int xs = (i & 1) ? CS + 1 - us : us;
+                        const uint32_t bs = smem_u32(smem + C::OFF_BR + (xs * C::P + tile) * C::BR_BYTES);
                         const uint32_t bd = smem_u32(smem + C::OFF_BD + tile * C::B_BYTES);
-                        const uint32_t dt = tmem + (uint32_t)(C::REV_COL + tile * C::NT);
+                        const uint32_t dt = tmem + (uint32_t)(C::REV_COL + tile * C::R);
 #pragma unroll
                         for (int ks = 0; ks < V / 16; ++ks)
                             tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
                                           smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
                                           ks > 0 ? 1u : 0u);
 #pragma unroll
+                        for (int ks = 0; ks < V / 16; ++ks)   // lo rows R .. 2R-1 of the dA operand
+                            tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
+                                          smem_desc(bd + (C::R / 8) * 128 + ks * 2 * C::NT * 16, C::NT * 16, 128),
+                                          idesc_g, 1u);
+#pragma unroll
                         for (int ks = 0; ks < C::R / 16; ++ks)
-                            tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::NT * 16),
+                            tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::R * 16),
                                           smem_desc(bd + ks * 256, 128, C::NT * 16), idesc_w,
                                           (first_dw && ks == 0) ? 0u : 1u);
                         first_dw = false;
@@ -673,12 +667,13 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                         ++nbr[tile];
                         tc_fence_after();
                         const uint32_t af = smem_u32(smem + C::OFF_AF + tile * C::AX_BYTES);
-                        const uint32_t br = smem_u32(smem + C::OFF_BR + tile * C::B_BYTES);
-                        const uint32_t dt = tmem + (uint32_t)(C::REC_COL + tile * C::NT);
+                        const int xs = (i & 1) ? CS + 1 - u : u;   // the epilogue's ring slot of H_{c0+u}
+                        const uint32_t br = smem_u32(smem + C::OFF_BR + (xs * C::P + tile) * C::BR_BYTES);
+                        const uint32_t dt = tmem + (uint32_t)(C::REC_COL + tile * C::R);
 #pragma unroll
                         for (int ks = 0; ks < V / 16; ++ks)
                             tc_mma_f16_ss(dt, smem_desc(af + ks * 256, 128, V * 16),
-                                          smem_desc(br + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_f,
+                                          smem_desc(br + ks * 2 * C::R * 16, C::R * 16, 128), idesc_f,
                                           ks > 0 ? 1u : 0u);
                         tc_commit(accfull_rec(tile));
                         issued[tile] = (int)(nbr[tile] - 1);
@@ -772,24 +767,30 @@ namespace {
 // Shapes of this file's kernel (the extended operands need V = 64 and tiles
 // of at least 16 rows); every other shape goes to the general-shape kernel of
 // bwd_tcg.cu.
+// The checkpoint stride is bounded by the tensor-memory scratch: 8 steps for
+// 64-row slices, 16 for 32-row ones.
 bool bwd_tcx_supported(int K, int V, int C) {
-    return V == 64 && (K == 32 || K == 64 || K == 128) && C >= 1 && C <= BwdTcCfg<64, 1>::CMAX;
+    if (V != 64 || C < 1) return false;
+    if (K == 32) return C <= BwdTcCfg<32, 1>::CMAX;
+    if (K == 64) return C <= BwdTcCfg<64, 1>::CMAX;
+    if (K == 128) return C <= BwdTcCfg<64, 2>::CMAX;
+    return false;
 }
 }  // namespace
 
-int bwd_tc_slices(int K, int V) {
-    if (bwd_tcx_supported(K, V, 1)) return K > 64 ? 2 : 1;
+int bwd_tc_slices(int K, int V, int C) {
+    if (bwd_tcx_supported(K, V, C)) return K > 64 ? 2 : 1;
     return bwd_tcg_slices(K, V);
 }
 
 bool bwd_tc_supported(int K, int V, int C) { return bwd_tcx_supported(K, V, C) || bwd_tcg_supported(K, V, C); }
 
-// Per (b, h): dW partials of each slice, and the recompute scratch of
-// 2·C·K·V values (C states and C Z's of a chunk).
+// Per (b, h): the dW partials of each slice (the recompute scratch lives in
+// tensor memory).
 size_t bwd_tc_workspace(int B, int H, int T, int K, int V, int C) {
     if (!bwd_tcx_supported(K, V, C)) return bwd_tcg_workspace(B, H, T, K, V, C);
-    const size_t nsl = (size_t)bwd_tc_slices(K, V);
-    return sizeof(float) * ((size_t)B * H * nsl * V * V + (size_t)B * H * 2 * C * K * V);
+    const size_t nsl = (size_t)bwd_tc_slices(K, V, C);
+    return sizeof(float) * (size_t)B * H * nsl * V * V;
 }
 
 cudaError_t launch_bwd_tc(const Params& p, cudaStream_t s) {

@@ -47,8 +47,9 @@ cudaError_t launch_bwd_tcg(const Params& p, cudaStream_t s);
 int fwd_tc_slices(int B, int H, int K, int V);
 // SMs of a B200 (the only target); used to decide when rows are sliced.
 constexpr int kNumSMs = 148;
-// Row slices (CTAs per (b, h)) of the tensor-core backward for a K x V state.
-int bwd_tc_slices(int K, int V);
+// Row slices (CTAs per (b, h)) of the tensor-core backward for a K x V state
+// and checkpoint stride C.
+int bwd_tc_slices(int K, int V, int C);
 
 // Workspace bytes beyond the 256-byte status header.
 size_t bwd_fp32_workspace(int B, int H, int K, int V, int C);

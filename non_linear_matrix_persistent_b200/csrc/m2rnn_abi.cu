@@ -150,7 +150,7 @@ m2rnn_status m2rnn_backward(const m2rnn_dims* d, const void* k, const void* v, c
     p.dy = dy; p.dHT = dHT; p.dk = dk; p.dv = dv; p.dq = dq; p.df = df; p.dW = dW; p.dH0 = dH0;
     uint8_t* extra = static_cast<uint8_t*>(workspace) + kStatusBytes;
     p.dW_part = reinterpret_cast<float*>(extra);
-    p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K, d->V);
+    p.dw_parts = d->mode == M2RNN_MODE_FP32_DEBUG ? 1 : m2rnn::bwd_tc_slices(d->K, d->V, d->ckpt_stride);
     p.scratch = p.dW_part + (size_t)d->B * d->H * p.dw_parts * d->V * d->V;
     const bool grouped = qk_group_partial_bytes(d) != 0;
     if (grouped) {   // the kernels write per-head dk / dq here; the group sums go to dk, dq

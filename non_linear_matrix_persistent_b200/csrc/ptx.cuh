@@ -182,6 +182,24 @@ __device__ __forceinline__ void tmem_ld_32x32b<32>(uint32_t taddr, uint32_t (&r)
         : "r"(taddr));
 }
 
+// Tensor-memory stores, 32x32b.xN: thread i of the warp writes lane (base+i),
+// N consecutive 32-bit columns.  Asynchronous: tc_wait_st() orders them
+// before a later tcgen05.ld of the same thread.
+#define M2RNN_W4(a) "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3])
+template <int N>
+__device__ __forceinline__ void tmem_st_32x32b(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 4 || N == 8, "tmem_st_32x32b width");
+    if constexpr (N == 4) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), M2RNN_W4(r)
+                     : "memory");
+    } else {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                     M2RNN_W4(r), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                     : "memory");
+    }
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 template <int N, int SPLIT>
 __device__ __forceinline__ void tmem_ld_16x32bx2(uint32_t taddr, uint32_t (&r)[N]) {
     static_assert(N == 4 || N == 8 || N == 16 || N == 32, "tmem_ld_16x32bx2 width");

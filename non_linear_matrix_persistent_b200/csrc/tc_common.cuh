@@ -85,9 +85,10 @@ __device__ __forceinline__ void write_state_operand(uint8_t* Bt, const float (&h
 
 // Writes only the hi parts (bf16, round to nearest) of this thread's RT
 // values of column j, at n = nloc + r: for operands whose lo half no MMA reads.
-template <class C>
+// NB: rows of the buffer (the same layout with NB in place of NT).
+template <class C, int NB = C::NT>
 __device__ __forceinline__ void write_state_operand_hi(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
-    uint8_t* colbase = Bt + (j >> 3) * (C::NT * 16) + (j & 7) * 16;
+    uint8_t* colbase = Bt + (j >> 3) * (NB * 16) + (j & 7) * 16;
     auto pack = [](float a, float b) {
         const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
         return *reinterpret_cast<const uint32_t*>(&v);
@@ -102,6 +103,27 @@ __device__ __forceinline__ void write_state_operand_hi(uint8_t* Bt, const float 
     } else {
         const uint2 hi = make_uint2(pack(h[0], h[1]), pack(h[2], h[3]));
         *reinterpret_cast<uint2*>(colbase + (nloc >> 3) * 128 + (nloc & 7) * 2) = hi;
+    }
+}
+
+// Reads back this thread's RT values of column j (as fp32) from an operand
+// written by write_state_operand_hi<C, NB> with the same j and nloc.
+template <class C, int NB = C::NT>
+__device__ __forceinline__ void read_state_operand_hi(const uint8_t* Bt, int j, int nloc, float (&h)[C::RT]) {
+    const uint8_t* colbase = Bt + (j >> 3) * (NB * 16) + (j & 7) * 16;
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g) {
+            const uint4 w = *reinterpret_cast<const uint4*>(colbase + ((nloc + 8 * g) >> 3) * 128);
+            h[8 * g + 0] = bf16lo_to_f32(w.x); h[8 * g + 1] = bf16hi_to_f32(w.x);
+            h[8 * g + 2] = bf16lo_to_f32(w.y); h[8 * g + 3] = bf16hi_to_f32(w.y);
+            h[8 * g + 4] = bf16lo_to_f32(w.z); h[8 * g + 5] = bf16hi_to_f32(w.z);
+            h[8 * g + 6] = bf16lo_to_f32(w.w); h[8 * g + 7] = bf16hi_to_f32(w.w);
+        }
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(colbase + (nloc >> 3) * 128 + (nloc & 7) * 2);
+        h[0] = bf16lo_to_f32(w.x); h[1] = bf16hi_to_f32(w.x);
+        h[2] = bf16lo_to_f32(w.y); h[3] = bf16hi_to_f32(w.y);
     }
 }
 

@@ -48,6 +48,7 @@ class Workload:
     seed: int = 0
     qk_heads: int = 0           # k / q head groups G (0: one per head)
     gate_logits: bool = False   # f holds the gate logit z + gate_shift instead of its sigmoid
+    ckpt_stride: int = 8        # checkpoint stride C of a training workload's forward and backward
 
     @property
     def tokens(self) -> int:
@@ -69,7 +70,7 @@ WORKLOADS: Dict[str, Workload] = {
                                 backward=True),
     # the 7B-MoE layer shape trained: its inputs plus dY ~ N(0, 1)
     "layer7b_moe_train": Workload("layer7b_moe_train", B=4, H=32, T=4096, K=128, V=128,
-                                  gate_var=1.5, gate_shift=1.5, backward=True),
+                                  gate_var=1.5, gate_shift=1.5, backward=True, ckpt_stride=16),
 }
 
 

@@ -102,10 +102,13 @@ def test_backward_argument_errors(L):
 
 def test_tc_backward_every_shape_has_a_workspace(L):
     """The tensor-core backward takes every K, V in {16, 32, 64, 128} with a
-    checkpoint stride of at most 16.  V = 64 with K >= 32 keeps the
-    extended-operand kernel's workspace (dW partials + 2·C·K·V scratch per
-    pair); K = 128 at V = 128 runs four 32-row slices per pair, whose dv and
-    df partials (4·B·H·T·(V + 1) fp32) are summed after the kernel."""
+    checkpoint stride of at most 16.  V = 64 with K >= 32 and a stride within
+    the extended-operand kernel's tensor-memory scratch (8 steps for K >= 64,
+    16 for K = 32) needs only the dW partials (one per 64-row slice); longer
+    strides there, and the other shapes, take the general-shape kernel, whose
+    workspace adds 2·C·KS·MX scratch values per CTA; K = 128 at V = 128 runs
+    four 32-row slices per pair, whose dv and df partials
+    (4·B·H·T·(V + 1) fp32) are summed after the kernel."""
     B, H, T, C = 2, 3, 5, 4
     for K in (16, 32, 64, 128):
         for V in (16, 32, 64, 128):
@@ -117,8 +120,13 @@ def test_tc_backward_every_shape_has_a_workspace(L):
             assert st == _lib.ERR_UNSUPPORTED_SHAPE, (K, V)
     def pad(n):
         return 256 + (n + 255) // 256 * 256
-    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=64, V=64, C=C), 1) == pad(
-        4 * (B * H * 64 * 64 + B * H * 2 * C * 64 * 64))
+    for K, cmax, nsl in ((32, 16, 1), (64, 8, 1), (128, 8, 2)):
+        for C in (1, 4, cmax):
+            assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=K, V=64, C=C), 1) == pad(
+                4 * B * H * nsl * 64 * 64), (K, C)
+    # K = V = 64 beyond 8 steps: the general-shape kernel (one 64-row slice, MX = 64)
+    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=64, V=64, C=12), 1) == pad(
+        4 * (B * H * 64 * 64 + 2 * 12 * B * H * 64 * 64))
     ncta = B * H * 4
     assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=128, V=128, C=C), 1) == pad(
         4 * (ncta * 128 * 128 + 2 * C * ncta * 32 * 128 + 4 * B * H * T * 129))

@@ -14,12 +14,15 @@ def test_per_step_counts_training_workload():
     K = V = 64
     assert fwd["flop"] == 2 * K * V * V and bwd["flop"] == 3 * 2 * K * V * V
     assert fwd["tanh"] == bwd["tanh"] == K * V
-    # forward: k, q, v bf16 in, f in, y fp32 out, the fp32 checkpoint every 16 steps
-    assert fwd["bytes"] == (2 * K + V) * 2 + 4 + 4 * V + 4 * K * V / 16 == 1668
-    # backward: k, q, v, dy bf16 and f in, dk, dq, dv, df fp32 out, one checkpoint read per 16 steps
-    assert bwd["bytes"] == (2 * K + 2 * V) * 2 + 4 + (2 * K + V) * 4 + 4 + 4 * K * V / 16 == 2312
+    assert WORKLOADS["layer410m_train"].ckpt_stride == 8
+    # forward: k, q, v bf16 in, f in, y fp32 out, the fp32 checkpoint every 8 steps
+    assert fwd["bytes"] == (2 * K + V) * 2 + 4 + 4 * V + 4 * K * V / 8 == 2692
+    # backward: k, q, v, dy bf16 and f in, dk, dq, dv, df fp32 out, one checkpoint read per 8 steps
+    assert bwd["bytes"] == (2 * K + 2 * V) * 2 + 4 + (2 * K + V) * 4 + 4 + 4 * K * V / 8 == 3336
     f_only, _ = bench.per_step_counts(WORKLOADS["layer410m_fwd"])
-    assert f_only["bytes"] == 1668 - 4 * K * V / 16   # no checkpoints without a backward
+    assert f_only["bytes"] == 2692 - 4 * K * V / 8   # no checkpoints without a backward
+    _, bwd7 = bench.per_step_counts(WORKLOADS["layer7b_moe_train"])
+    assert bwd7["bytes"] == (4 * 128) * 2 + 4 + (3 * 128) * 4 + 4 + 4 * 128 * 128 / 16
 
 
 def test_kernel_digest_ignores_comments_only():
@@ -149,3 +152,7 @@ def test_backward_kernel_rule():
     assert bench.backward_kernel(w) == ("m2rnn_bwd_tc_kernel", "bwd_tc.cu")
     assert bench.backward_kernel(WORKLOADS["layer7b_moe_train"]) == ("m2rnn_bwd_tcg_kernel", "bwd_tcg.cu")
     assert bench.backward_kernel(w.with_(K=16)) == ("m2rnn_bwd_tcg_kernel", "bwd_tcg.cu")
+    # the extended-operand kernel's scratch holds 8 steps at K = 64, 128 and 16 at K = 32
+    assert bench.backward_kernel(w.with_(ckpt_stride=16)) == ("m2rnn_bwd_tcg_kernel", "bwd_tcg.cu")
+    assert bench.backward_kernel(w.with_(K=128)) == ("m2rnn_bwd_tc_kernel", "bwd_tc.cu")
+    assert bench.backward_kernel(w.with_(K=32, ckpt_stride=16)) == ("m2rnn_bwd_tc_kernel", "bwd_tc.cu")

@@ -195,7 +195,7 @@ def _spectral_radii(W):
 
 def test_train_workload_several_heads_per_pair():
     """The full training workload (B=8, H=16, K=V=64, T=2048; forward with
-    checkpoints every 16 steps, then the backward) in the benchmark's launch
+    checkpoints every 8 steps, then the backward) in the benchmark's launch
     configuration.  Three whole heads are checked against the oracle: the
     head whose W has the largest spectral radius (the most sensitive
     recurrence), the one with the smallest, and head 5.  Every (b, h) pair's
@@ -205,8 +205,9 @@ def test_train_workload_several_heads_per_pair():
     x = make_inputs(w)
     xc = _cuda(x)
     a = api()
-    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=16, want_ckpt=True)
-    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=16)
+    C = w.ckpt_stride
+    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True)
+    g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], ckpt_stride=C)
     torch.cuda.synchronize()
     assert a.device_status() == 0
     rho = _spectral_radii(x["W"])

@@ -441,7 +441,7 @@ def test_train_workload_sampled_head():
     w = WORKLOADS["layer410m_train"]
     x = make_inputs(w)
     xc = _cuda(x)
-    g = _gpu_fwd_bwd(xc, 16)
+    g = _gpu_fwd_bwd(xc, w.ckpt_stride)
     for n, t in g.items():
         assert torch.isfinite(t).all(), n
     h = 5
@@ -460,7 +460,7 @@ def test_train_7b_moe_shape_sampled_head():
     w = WORKLOADS["layer7b_moe_train"]
     x = make_inputs(w)
     xc = _cuda(x)
-    g = _gpu_fwd_bwd(xc, 16)
+    g = _gpu_fwd_bwd(xc, w.ckpt_stride)
     for n, t in g.items():
         assert torch.isfinite(t).all(), n
     h = 11
