@@ -159,6 +159,44 @@ __device__ __forceinline__ int ag_off(int m, int k) {
     return (k >> 3) * (128 * 16) + (m >> 3) * 128 + (k & 7) * 16 + (m & 7) * 2;
 }
 
+// The bf16 state values (round to nearest) of one thread's RT rows of its
+// column in a state operand, at the thread's own position tp within it:
+// tp = operand + (j/8)·(R·16) + (j%8)·16 + (nloc/8)·128 + (nloc%8)·2, the
+// layout of write_state_operand_hi<C, R> (the next 8-row group 128 bytes on).
+template <class C>
+__device__ __forceinline__ void put_state_hi(uint8_t* tp, const float (&h)[C::RT]) {
+    auto pack = [](float a, float b) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&v);
+    };
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g)
+            *reinterpret_cast<uint4*>(tp + g * 128) =
+                make_uint4(pack(h[8 * g], h[8 * g + 1]), pack(h[8 * g + 2], h[8 * g + 3]),
+                           pack(h[8 * g + 4], h[8 * g + 5]), pack(h[8 * g + 6], h[8 * g + 7]));
+    } else {
+        *reinterpret_cast<uint2*>(tp) = make_uint2(pack(h[0], h[1]), pack(h[2], h[3]));
+    }
+}
+template <class C>
+__device__ __forceinline__ void get_state_hi(const uint8_t* tp, float (&h)[C::RT]) {
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g) {
+            const uint4 w = *reinterpret_cast<const uint4*>(tp + g * 128);
+            h[8 * g + 0] = bf16lo_to_f32(w.x); h[8 * g + 1] = bf16hi_to_f32(w.x);
+            h[8 * g + 2] = bf16lo_to_f32(w.y); h[8 * g + 3] = bf16hi_to_f32(w.y);
+            h[8 * g + 4] = bf16lo_to_f32(w.z); h[8 * g + 5] = bf16hi_to_f32(w.z);
+            h[8 * g + 6] = bf16lo_to_f32(w.w); h[8 * g + 7] = bf16hi_to_f32(w.w);
+        }
+    } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(tp);
+        h[0] = bf16lo_to_f32(w.x); h[1] = bf16hi_to_f32(w.x);
+        h[2] = bf16lo_to_f32(w.y); h[3] = bf16hi_to_f32(w.y);
+    }
+}
+
 // Stores the extra output row (TMEM lane XLANE) of one tile, its R columns,
 // to dst[0 .. R).  Warp-collective over lane quarter 0; thread XLANE stores,
 // and only when `store` is set.
@@ -293,8 +331,6 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // down, one step ahead) has already read.  Only the thread that wrote
         // a value reads it back.
         const uint32_t scr = tmem + lanes + (uint32_t)(C::SCR_COL + slot * C::RT);
-        auto sslot = [&](int i, int u) { return (i & 1) ? CS - 1 - u : u; };
-        auto scr_at = [&](int x) { return scr + (uint32_t)(x * C::SCR_STEP); };
         // State operands H_{c0+u} (bf16, round to nearest) in a ring of CS + 2
         // slots per tile: the recompute MMA of step c0+u reads slot x(u), and
         // so does, one phase later, the dW MMA of the same step.  The mirror
@@ -304,8 +340,11 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // its chunk from the top down while the recompute writes from the
         // bottom up; the dW MMA of reverse step s may run until reverse step
         // s+1 starts, one step after the epilogue's own reads).
-        auto bslot = [&](int i, int u) { return (i & 1) ? CS + 1 - u : u; };
-        auto Br = [&](int x) { return smem + C::OFF_BR + (x * C::P + tile) * C::BR_BYTES; };
+        // This thread's values in ring slot 0; slot x is x·RING_STEP bytes on.
+        constexpr int RING_STEP = C::P * C::BR_BYTES;
+        uint8_t* const brt = smem + C::OFF_BR + tile * C::BR_BYTES + (j >> 3) * (C::R * 16) + (j & 7) * 16 +
+                             (nloc >> 3) * 128 + (nloc & 7) * 2;
+
         auto stage = [&](int i) { return smem + C::OFF_RING + (i % C::NSTAGE) * C::STAGE_BYTES; };
 
         float G[C::RT], h[C::RT];
@@ -334,6 +373,17 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
             auto dyr = [&](int u) {   // dy of step c0r + u of the recompute chunk, u >= -1
                 return reinterpret_cast<const uint16_t*>(str + C::ST_DY + (u + 1) * V * 2);
             };
+            // Slots of chunk-local step u: the chunk recomputed in an even phase
+            // walks both slot sets upwards from slot 0, in an odd phase downwards
+            // from the last slot (scratch CS-1, ring CS+1); phase m recomputes
+            // with its own parity and reverses the chunk of phase m-1.
+            const bool odd = (m & 1) != 0;
+            uint8_t* const rec_ring = brt + (odd ? (CS + 1) * RING_STEP : 0);
+            uint8_t* const rev_ring = brt + (odd ? 0 : (CS + 1) * RING_STEP);
+            const int rec_rstep = odd ? -RING_STEP : RING_STEP;
+            const uint32_t rec_scr = scr + (uint32_t)(odd ? (CS - 1) * C::SCR_STEP : 0);
+            const uint32_t rev_scr = scr + (uint32_t)(odd ? 0 : (CS - 1) * C::SCR_STEP);
+            const int rec_sstep = odd ? -C::SCR_STEP : C::SCR_STEP;
 
             if (has_rev) {
                 const int i = m - 1;
@@ -344,8 +394,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 }
                 // before the recompute below stores its first step (same slot)
                 tc_wait_st();
-                tmem_ld_32x32b<C::RT>(scr_at(sslot(m - 1, lenv - 1)), sz);
-                read_state_operand_hi<C, C::R>(Br(bslot(m - 1, lenv - 1)), j, nloc, hp);
+                tmem_ld_32x32b<C::RT>(rev_scr - (uint32_t)((lenv - 1) * rec_sstep), sz);
+                get_state_hi<C>(rev_ring - (lenv - 1) * rec_rstep, hp);
             }
             if (has_rec) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(m % C::NSTAGE), (m / C::NSTAGE) & 1, abort_flag, p));
@@ -357,7 +407,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 for (int r = 0; r < C::RT; ++r) h[r] = ck[(row0 + r) * V + j];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ck_empty);
-                write_state_operand_hi<C, C::R>(Br(bslot(m, 0)), h, j, nloc);
+                put_state_hi<C>(rec_ring, h);
                 if (xwriter) *xf = c0r > 0 ? dyr(-1)[j] : (uint16_t)0;
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -413,8 +463,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 if (lane == 0) mbar_arrive(bready_rev(tile));
                 if (u > 0) {   // the next reverse step's operands, ahead of the recompute step that reuses the slot
                     tc_wait_st();
-                    tmem_ld_32x32b<C::RT>(scr_at(sslot(m - 1, u - 1)), sz);
-                    read_state_operand_hi<C, C::R>(Br(bslot(m - 1, u - 1)), j, nloc, hp);
+                    tmem_ld_32x32b<C::RT>(rev_scr - (uint32_t)((u - 1) * rec_sstep), sz);
+                    get_state_hi<C>(rev_ring - (u - 1) * rec_rstep, hp);
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
@@ -451,11 +501,11 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                         st[r] = __float_as_uint(z);
                         h[r] = fmaf(g, z - h[r], h[r]);
                     }
-                    tmem_st_32x32b<C::RT>(scr_at(sslot(m, u)), st);
+                    tmem_st_32x32b<C::RT>(rec_scr + (uint32_t)(u * rec_sstep), st);
                 }
                 tc_fence_before();
                 if (u + 1 < nmr) {
-                    write_state_operand_hi<C, C::R>(Br(bslot(m, u + 1)), h, j, nloc);
+                    put_state_hi<C>(rec_ring + (u + 1) * rec_rstep, h);
                     if (xwriter) *xf = dyr(u)[j];
                     fence_proxy_async_smem();
                     __syncwarp();
