@@ -33,9 +33,9 @@
 // cycles, and issue -> commit -> mbarrier wake-up adds ~400 cycles, so a
 // step is bound by that round trip plus the epilogue, not by tensor
 // throughput.  The state rows of a pair are therefore split into P = 2 tiles
-// whose chains run concurrently (ping-pong): while the epilogue warps of one
-// tile run tanh and the blend, the tensor core computes the other tile's
-// product.  Two warps per TMEM lane quarter serve each tile (when the tile
+// (4 at K = V = 128) whose chains run concurrently (ping-pong): while the
+// epilogue warps of one tile run tanh and the blend, the tensor core computes
+// another tile's product.  Two warps per TMEM lane quarter serve each tile (when the tile
 // has enough rows), so that each thread handles few rows.
 //
 // Warp roles: warps [0, P·WPT) epilogue (warp w serves tile w / WPT, TMEM
@@ -58,17 +58,23 @@
 
 namespace m2rnn {
 
-template <int K_, int V_>
+template <int K_, int V_, bool FAST_ = false>
 struct FwdTcCfg {
     static constexpr int K = K_, V = V_;
-    static constexpr int P = 2;
+    // row tiles with independent chains: 4 at K = V = 128 with the accurate
+    // tanh, where the epilogue (32 rows per thread) and the MMA (N = 128 per
+    // tile) are both long enough that two more chains in flight pay (8.86 ->
+    // 7.70 ms at B = 4, 32 heads, T = 4096, bit-identical results); 2
+    // elsewhere (the fast-tanh kernel at K = V = 128: 6.10 -> 7.34 ms with 4;
+    // four 16-row tiles at K = V = 64 measured 17% slower)
+    static constexpr int P = (V == 128 && K == 128 && !FAST_) ? 4 : 2;
     static constexpr int MPAD = V <= 64 ? 64 : 128;
     static constexpr int R = K / P;                       // state rows per tile
     static constexpr int NT = 2 * R;                      // MMA N per tile (hi rows, then lo rows)
     // row groups per tile served by separate warps of the same lane quarter,
     // so that each thread handles at most 16 rows (measured on B200 at
     // K = V = 64: 1.85 -> 1.75 ms per 2048-step scan of 128 (b, h) pairs)
-    static constexpr int SUBS = (MPAD == 128 || K >= 64) ? 2 : 1;
+    static constexpr int SUBS = P == 4 ? 1 : (MPAD == 128 || K >= 64) ? 2 : 1;
     static constexpr int WPT = 4 * SUBS;                  // epilogue warps per tile
     static constexpr int RT = (MPAD == 64) ? R / (2 * SUBS) : R / SUBS;  // rows per thread
     static constexpr int CH = RT < 16 ? RT : 16;          // rows per tensor-memory load
@@ -114,8 +120,8 @@ struct FwdTcCfg {
 // run-time test never fires without checkpoints; dropping that code altogether
 // measured slower at V = 128 (8.83 -> 9.15 ms) and equal at V = 64.
 template <int K, int V, bool FAST, bool CKPT>
-__global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
-    using C = FwdTcCfg<K, V>;
+__global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
+    using C = FwdTcCfg<K, V, FAST>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // One CTA per (b, h) and slice of K rows (p.slices slices of the p.K state
@@ -426,17 +432,23 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V>::NTHREADS, 1) m2rnn_fwd_tc_kern
     }
 }
 
-template <int K, int V>
-static cudaError_t launch_fwd_tc_kv(const Params& p, cudaStream_t stream) {
-    using C = FwdTcCfg<K, V>;
-    auto kern = p.ckpt != nullptr ? (p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true, true>
-                                                 : m2rnn_fwd_tc_kernel<K, V, false, true>)
-                                  : (p.fast_tanh ? m2rnn_fwd_tc_kernel<K, V, true, false>
-                                                 : m2rnn_fwd_tc_kernel<K, V, false, false>);
+template <int K, int V, bool FAST, bool CKPT>
+static cudaError_t launch_fwd_tc_one(const Params& p, cudaStream_t stream) {
+    using C = FwdTcCfg<K, V, FAST>;
+    auto kern = m2rnn_fwd_tc_kernel<K, V, FAST, CKPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<p.B * p.H * p.slices, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <int K, int V>
+static cudaError_t launch_fwd_tc_kv(const Params& p, cudaStream_t stream) {
+    if (p.ckpt != nullptr)
+        return p.fast_tanh ? launch_fwd_tc_one<K, V, true, true>(p, stream)
+                           : launch_fwd_tc_one<K, V, false, true>(p, stream);
+    return p.fast_tanh ? launch_fwd_tc_one<K, V, true, false>(p, stream)
+                       : launch_fwd_tc_one<K, V, false, false>(p, stream);
 }
 
 template <int K>
