@@ -34,8 +34,9 @@
 //
 // Layout: one CTA per (b, h) and slice of RS = 8 rows (4 row warps), plus a
 // bulk-copy producer warp (this slice's 8 values of k_t and q_t, the pair's
-// v_t, f_t for TC steps per ring stage) and a storer warp that sums the rows'
-// readout partials q_t[i]·h_t[i, :] in row order.  With several slices per
+// v_t, f_t for TC steps per ring stage) and a storer warp that sums the row
+// warps' readout partials (each warp's two rows q_t[i]·h_t[i, :] +
+// q_t[i+1]·h_t[i+1, :]) in warp order.  With several slices per
 // pair the slices' partial readouts go to the workspace and
 // m2rnn_y_reduce_kernel adds them in slice order.  Supported: V = 64 (W takes
 // 128 registers per lane) and at most 148 CTAs (one wave, one CTA per SM).
@@ -62,7 +63,7 @@ struct FwdRowsCfg {
     static constexpr int ST_V = 2 * TC * RS * 2;   // [TC][V] bf16
     static constexpr int ST_F = ST_V + TC * V * 2; // [TC] fp32
     static constexpr int STAGE_BYTES = ((ST_F + TC * 4) + 127) / 128 * 128;
-    static constexpr int YBUF_BYTES = TC * RS * V * 4;   // [TC][RS][V] readout partials
+    static constexpr int YBUF_BYTES = TC * NWR * V * 4;  // [TC][NWR][V] readout partials, one per row warp
     static constexpr int HROW_BYTES = 2 * RW * V * 4;    // per warp: its rows, double-buffered
     static constexpr int OFF_RING = 0;
     static constexpr int OFF_Y = OFF_RING + S * STAGE_BYTES;
@@ -195,8 +196,10 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             // readout partials of the two rows: q_t[i]·h_t[i, :]
             const uint32_t qq = *reinterpret_cast<const uint32_t*>(st + C::ST_Q + (tt * RS + r0) * 2);
             const float q0 = bf16lo_to_f32(qq), q1 = bf16hi_to_f32(qq);
-            float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * RS + r0) * V;
-            yb[j0] = q0 * h0.x; yb[j1] = q0 * h0.y; yb[V + j0] = q1 * h1.x; yb[V + j1] = q1 * h1.y;
+            // the warp's two rows summed here, so that the storer adds NWR partials
+            float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * C::NWR + warp) * V;
+            yb[j0] = fmaf(q1, h1.x, q0 * h0.x);
+            yb[j1] = fmaf(q1, h1.y, q0 * h0.y);
             if (CKPT && t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1}
                 ck_next += p.C;
                 ++ck_idx;
@@ -264,10 +267,10 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             float* yg = yout + ((size_t)bh * T + t0) * V;
             for (int e = lane * 4; e < nt * V; e += 128) {
                 const int tt = e / V, jj = e % V;
-                const float* src = yb + tt * RS * V + jj;
+                const float* src = yb + tt * C::NWR * V + jj;
                 float4 a = *reinterpret_cast<const float4*>(src);
 #pragma unroll
-                for (int r = 1; r < RS; ++r) {
+                for (int r = 1; r < C::NWR; ++r) {
                     const float4 b = *reinterpret_cast<const float4*>(src + r * V);
                     a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
                 }
