@@ -15,9 +15,10 @@
 // warp two state rows for all T steps instead, with W resident in registers,
 // so a step needs no block-level synchronisation at all: the warp shares its
 // two rows through shared memory (__syncwarp), every lane reads both rows in
-// 16-byte broadcast loads, and lane l forms columns l and l + 32 of each row's
-// product h_{t-1}·W with packed FFMA2 (W[l'][l], W[l'][l + 32] as fp32 pairs,
-// 64 of them, shared by the two rows) in four accumulator chains per row.
+// 16-byte broadcast loads, and lane l forms columns 2l and 2l + 1 of each
+// row's product h_{t-1}·W with packed FFMA2 (W[l'][2l], W[l'][2l + 1] as fp32
+// pairs, 64 of them, shared by the two rows) in four accumulator chains per
+// row; a lane's two adjacent columns move in 8-byte accesses.
 // Measured on B200 at the long B = 1 workload (1,024 rows on 128 SMs): one
 // row per warp 8.1 ms, two rows per warp (this kernel) 6.2 ms; slower were
 // the same with the h row stored as duplicated pairs (7.9 ms), a row pair
@@ -119,21 +120,24 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
         // ------------------------------------------------------------ two state rows per warp
         const int r0 = warp * 2;                   // first row of this warp within the slice
         const int i = koff + r0;                   // its state row
-        const int j0 = lane, j1 = lane + 32;       // state columns of this lane
-        // W columns j0, j1 as fp32 pairs, resident for all T steps
+        const int j0 = 2 * lane;                   // state columns j0, j0 + 1 of this lane (8-byte accesses)
+        // W columns j0, j0 + 1 as fp32 pairs, resident for all T steps
         float2 Wr[V];
         {
             const uint16_t* Wg = static_cast<const uint16_t*>(p.W) + (size_t)hd * V * V;
 #pragma unroll
-            for (int l = 0; l < V; ++l)
-                Wr[l] = make_float2(bf16lo_to_f32(Wg[l * V + j0]), bf16lo_to_f32(Wg[l * V + j1]));
+            for (int l = 0; l < V; ++l) {
+                const uint32_t w2 = *reinterpret_cast<const uint32_t*>(Wg + l * V + j0);
+                Wr[l] = make_float2(bf16lo_to_f32(w2), bf16hi_to_f32(w2));
+            }
         }
         const size_t srow0 = ((size_t)bh * K + i) * V, srow1 = srow0 + V;
-        float2 h0 = p.H0 != nullptr ? make_float2(p.H0[srow0 + j0], p.H0[srow0 + j1]) : make_float2(0.f, 0.f);
-        float2 h1 = p.H0 != nullptr ? make_float2(p.H0[srow1 + j0], p.H0[srow1 + j1]) : make_float2(0.f, 0.f);
+        float2 h0 = p.H0 != nullptr ? *reinterpret_cast<const float2*>(p.H0 + srow0 + j0) : make_float2(0.f, 0.f);
+        float2 h1 = p.H0 != nullptr ? *reinterpret_cast<const float2*>(p.H0 + srow1 + j0) : make_float2(0.f, 0.f);
         if (CKPT) {
             float* ck = p.ckpt + (size_t)bh * nck * K * V + (size_t)i * V;
-            ck[j0] = h0.x; ck[j1] = h0.y; ck[V + j0] = h1.x; ck[V + j1] = h1.y;
+            *reinterpret_cast<float2*>(ck + j0) = h0;
+            *reinterpret_cast<float2*>(ck + V + j0) = h1;
         }
         float* hrow = reinterpret_cast<float*>(smem + C::OFF_H + warp * C::HROW_BYTES);
         // next checkpoint step as a running count (no per-step remainder by the run-time stride)
@@ -153,12 +157,14 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             // every lane read this one at step t-2 before it reached the
             // __syncwarp of step t-1, which this lane has passed.
             float* hb = hrow + (t & 1) * 2 * V;
-            hb[j0] = h0.x; hb[j1] = h0.y; hb[V + j0] = h1.x; hb[V + j1] = h1.y;
+            *reinterpret_cast<float2*>(hb + j0) = h0;
+            *reinterpret_cast<float2*>(hb + V + j0) = h1;
             __syncwarp();
             const uint32_t kk = *reinterpret_cast<const uint32_t*>(st + C::ST_K + (tt * RS + r0) * 2);
             const uint16_t* vt = reinterpret_cast<const uint16_t*>(st + C::ST_V + tt * V * 2);
-            const float2 v2 = make_float2(bf16lo_to_f32(vt[j0]), bf16lo_to_f32(vt[j1]));
-            // h_{t-1}·W[:, (j0, j1)] for both rows: four accumulator chains per row over l mod 4
+            const uint32_t vv = *reinterpret_cast<const uint32_t*>(vt + j0);
+            const float2 v2 = make_float2(bf16lo_to_f32(vv), bf16hi_to_f32(vv));
+            // h_{t-1}·W[:, (j0, j0 + 1)] for both rows: four accumulator chains per row over l mod 4
             float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0, b0 = a0, b1 = a0, b2 = a0, b3 = a0;
             const float4* hb4 = reinterpret_cast<const float4*>(hb);
 #pragma unroll
@@ -198,14 +204,14 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             const float q0 = bf16lo_to_f32(qq), q1 = bf16hi_to_f32(qq);
             // the warp's two rows summed here, so that the storer adds NWR partials
             float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES) + (tt * C::NWR + warp) * V;
-            yb[j0] = fmaf(q1, h1.x, q0 * h0.x);
-            yb[j1] = fmaf(q1, h1.y, q0 * h0.y);
+            *reinterpret_cast<float2*>(yb + j0) = make_float2(fmaf(q1, h1.x, q0 * h0.x), fmaf(q1, h1.y, q0 * h0.y));
             if (CKPT && t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1}
                 ck_next += p.C;
                 ++ck_idx;
                 if ((t + 1) < T) {
                     float* ck = p.ckpt + ((size_t)bh * nck + ck_idx) * K * V + (size_t)i * V;
-                    ck[j0] = h0.x; ck[j1] = h0.y; ck[V + j0] = h1.x; ck[V + j1] = h1.y;
+                    *reinterpret_cast<float2*>(ck + j0) = h0;
+                    *reinterpret_cast<float2*>(ck + V + j0) = h1;
                 }
             }
             if (tt == C::TC - 1 || t == T - 1) {
@@ -217,7 +223,8 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             }
         }
         if (ok && p.HT != nullptr) {
-            p.HT[srow0 + j0] = h0.x; p.HT[srow0 + j1] = h0.y; p.HT[srow1 + j0] = h1.x; p.HT[srow1 + j1] = h1.y;
+            *reinterpret_cast<float2*>(p.HT + srow0 + j0) = h0;
+            *reinterpret_cast<float2*>(p.HT + srow1 + j0) = h1;
         }
     } else if (warp == C::W_PROD) {
         // ------------------------------------------------------------ producer
