@@ -268,6 +268,28 @@ __device__ __forceinline__ float tanh_exp(float x) {
     const float e = __expf(2.f * x);
     return 1.f - __fdividef(2.f, 1.f + e);
 }
+// tanh of two values from the identity tanh(x) = 1 - 2 / (1 + 2^{x·2/ln 2}),
+// with the hardware base-2 exponential and reciprocal approximations
+// (ex2.approx.ftz.f32, rcp.approx.ftz.f32: two SFU operations per value, as
+// in tanh_exp) and the surrounding arithmetic on packed fp32 pairs.  For
+// large |x| the exponential meets 0 or +inf, and the result is exactly -1 or
+// +1.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 tanh2_ex2(float2 x) {
+    constexpr float kTwoOverLn2 = 2.885390081777927f;   // 2 / ln 2 = 2 log2(e)
+    const float2 y = __fmul2_rn(x, make_float2(kTwoOverLn2, kTwoOverLn2));
+    const float2 d = __fadd2_rn(make_float2(ex2_approx(y.x), ex2_approx(y.y)), make_float2(1.f, 1.f));
+    return __ffma2_rn(make_float2(-2.f, -2.f), make_float2(rcp_approx(d.x), rcp_approx(d.y)), make_float2(1.f, 1.f));
+}
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
