@@ -134,88 +134,88 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
         int ck_next = p.ckpt != nullptr ? p.C : T + 1, ck_idx = 0;
 
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int c = t / C::TC, tt = t - c * C::TC, s = c % C::S;
+        // one chunk of TC steps per outer iteration: the ring and readout waits
+        // and arrivals stay out of the step loop, whose body is one straight block
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const int s = c % C::S, nt = min(C::TC, T - c * C::TC);
             const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
-            if (tt == 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (c / C::S) & 1, abort_flag, p));
-                if (ok && c >= 2)
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
-                if (!ok) break;
-            }
-            // H_{t-1} W: the state as compensated hi + lo bf16 A fragments
-            float acc[C::NT8][4];
-#pragma unroll
-            for (int nt = 0; nt < C::NT8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ++ks) {
-                uint32_t ahi[4], alo[4];
-                split_pack(h[2 * ks][0], h[2 * ks][1], ahi[0], alo[0]);
-                split_pack(h[2 * ks][2], h[2 * ks][3], ahi[1], alo[1]);
-                split_pack(h[2 * ks + 1][0], h[2 * ks + 1][1], ahi[2], alo[2]);
-                split_pack(h[2 * ks + 1][2], h[2 * ks + 1][3], ahi[3], alo[3]);
-#pragma unroll
-                for (int nt = 0; nt < C::NT8; ++nt) {
-                    mma_bf16_16816(acc[nt], ahi, wb[ks][nt][0], wb[ks][nt][1]);
-                    mma_bf16_16816(acc[nt], alo, wb[ks][nt][0], wb[ks][nt][1]);
-                }
-            }
-            // rank-1 term, tanh, gate blend
-            const uint16_t* kt = reinterpret_cast<const uint16_t*>(st + C::ST_K + tt * K * 2);
-            const uint16_t* qt = reinterpret_cast<const uint16_t*>(st + C::ST_Q + tt * K * 2);
-            const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + C::ST_V + tt * V * 2);
-            const float gt = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
-            const float k0 = bf16lo_to_f32(kt[i0]), k1 = bf16lo_to_f32(kt[i1]);
-#pragma unroll
-            for (int nt = 0; nt < C::NT8; ++nt) {
-                const uint32_t vv = vt[4 * nt + tq];   // v[8nt + 2tq], v[8nt + 2tq + 1]
-                const float v0 = bf16lo_to_f32(vv), v1 = bf16hi_to_f32(vv);
-                const float a0 = fmaf(k0, v0, acc[nt][0]), a1 = fmaf(k0, v1, acc[nt][1]);
-                const float a2 = fmaf(k1, v0, acc[nt][2]), a3 = fmaf(k1, v1, acc[nt][3]);
-                h[nt][0] = fmaf(gt, tanh_exp(a0) - h[nt][0], h[nt][0]);
-                h[nt][1] = fmaf(gt, tanh_exp(a1) - h[nt][1], h[nt][1]);
-                h[nt][2] = fmaf(gt, tanh_exp(a2) - h[nt][2], h[nt][2]);
-                h[nt][3] = fmaf(gt, tanh_exp(a3) - h[nt][3], h[nt][3]);
-            }
-            // readout partial over this warp's 16 rows: per column, q_i0 H[i0] + q_i1 H[i1],
-            // then a reduce-scatter over the 8 lanes of a column group (lane bits 2-4)
-            // that leaves lane (g, tq) with columns 8g + 2tq and 8g + 2tq + 1
-            {
-                const float q0 = bf16lo_to_f32(qt[i0]), q1 = bf16lo_to_f32(qt[i1]);
-                float pr[2 * C::NT8];
-#pragma unroll
-                for (int nt = 0; nt < C::NT8; ++nt) {
-                    pr[2 * nt] = fmaf(q1, h[nt][2], q0 * h[nt][0]);
-                    pr[2 * nt + 1] = fmaf(q1, h[nt][3], q0 * h[nt][1]);
-                }
-#pragma unroll
-                for (int lvl = 0; lvl < 3; ++lvl) {
-                    const int m = 16 >> lvl, n = 16 >> lvl;   // lane mask; live values 16, 8, 4
-                    const bool up = (lane & m) != 0;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (i < n / 2) {
-                            const float send = up ? pr[i] : pr[i + n / 2];
-                            const float keep = up ? pr[i + n / 2] : pr[i];
-                            pr[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-                        }
+            ok = __all_sync(0xffffffffu, mbar_wait_bounded(in_full(s), (c / C::S) & 1, abort_flag, p));
+            if (ok && c >= 2)
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
+            if (!ok) break;
+            for (int tt = 0; tt < nt; ++tt) {
+                const int t = c * C::TC + tt;
+                // H_{t-1} W: the state as compensated hi + lo bf16 A fragments
+                float acc[C::NT8][4];
+    #pragma unroll
+                for (int nt = 0; nt < C::NT8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    #pragma unroll
+                for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                    uint32_t ahi[4], alo[4];
+                    split_pack(h[2 * ks][0], h[2 * ks][1], ahi[0], alo[0]);
+                    split_pack(h[2 * ks][2], h[2 * ks][3], ahi[1], alo[1]);
+                    split_pack(h[2 * ks + 1][0], h[2 * ks + 1][1], ahi[2], alo[2]);
+                    split_pack(h[2 * ks + 1][2], h[2 * ks + 1][3], ahi[3], alo[3]);
+    #pragma unroll
+                    for (int nt = 0; nt < C::NT8; ++nt) {
+                        mma_bf16_16816(acc[nt], ahi, wb[ks][nt][0], wb[ks][nt][1]);
+                        mma_bf16_16816(acc[nt], alo, wb[ks][nt][0], wb[ks][nt][1]);
                     }
                 }
-                float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES);
-                *reinterpret_cast<float2*>(yb + (warp * C::TC + tt) * V + 8 * g + 2 * tq) = make_float2(pr[0], pr[1]);
-            }
-            if (t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1} (ck_next lies past T without checkpoints)
-                ck_next += p.C;
-                ++ck_idx;
-                if ((t + 1) < T) store_state(p.ckpt + ((size_t)bh * nck + ck_idx) * K * V);
-            }
-            if (tt == C::TC - 1 || t == T - 1) {
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(in_empty(s));
-                    mbar_arrive(ypfull(c & 1));
+                // rank-1 term, tanh, gate blend
+                const uint16_t* kt = reinterpret_cast<const uint16_t*>(st + C::ST_K + tt * K * 2);
+                const uint16_t* qt = reinterpret_cast<const uint16_t*>(st + C::ST_Q + tt * K * 2);
+                const uint32_t* vt = reinterpret_cast<const uint32_t*>(st + C::ST_V + tt * V * 2);
+                const float gt = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
+                const float k0 = bf16lo_to_f32(kt[i0]), k1 = bf16lo_to_f32(kt[i1]);
+    #pragma unroll
+                for (int nt = 0; nt < C::NT8; ++nt) {
+                    const uint32_t vv = vt[4 * nt + tq];   // v[8nt + 2tq], v[8nt + 2tq + 1]
+                    const float v0 = bf16lo_to_f32(vv), v1 = bf16hi_to_f32(vv);
+                    const float a0 = fmaf(k0, v0, acc[nt][0]), a1 = fmaf(k0, v1, acc[nt][1]);
+                    const float a2 = fmaf(k1, v0, acc[nt][2]), a3 = fmaf(k1, v1, acc[nt][3]);
+                    h[nt][0] = fmaf(gt, tanh_exp(a0) - h[nt][0], h[nt][0]);
+                    h[nt][1] = fmaf(gt, tanh_exp(a1) - h[nt][1], h[nt][1]);
+                    h[nt][2] = fmaf(gt, tanh_exp(a2) - h[nt][2], h[nt][2]);
+                    h[nt][3] = fmaf(gt, tanh_exp(a3) - h[nt][3], h[nt][3]);
                 }
+                // readout partial over this warp's 16 rows: per column, q_i0 H[i0] + q_i1 H[i1],
+                // then a reduce-scatter over the 8 lanes of a column group (lane bits 2-4)
+                // that leaves lane (g, tq) with columns 8g + 2tq and 8g + 2tq + 1
+                {
+                    const float q0 = bf16lo_to_f32(qt[i0]), q1 = bf16lo_to_f32(qt[i1]);
+                    float pr[2 * C::NT8];
+    #pragma unroll
+                    for (int nt = 0; nt < C::NT8; ++nt) {
+                        pr[2 * nt] = fmaf(q1, h[nt][2], q0 * h[nt][0]);
+                        pr[2 * nt + 1] = fmaf(q1, h[nt][3], q0 * h[nt][1]);
+                    }
+    #pragma unroll
+                    for (int lvl = 0; lvl < 3; ++lvl) {
+                        const int m = 16 >> lvl, n = 16 >> lvl;   // lane mask; live values 16, 8, 4
+                        const bool up = (lane & m) != 0;
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            if (i < n / 2) {
+                                const float send = up ? pr[i] : pr[i + n / 2];
+                                const float keep = up ? pr[i + n / 2] : pr[i];
+                                pr[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                            }
+                        }
+                    }
+                    float* yb = reinterpret_cast<float*>(smem + C::OFF_Y + (c & 1) * C::YBUF_BYTES);
+                    *reinterpret_cast<float2*>(yb + (warp * C::TC + tt) * V + 8 * g + 2 * tq) = make_float2(pr[0], pr[1]);
+                }
+                if (t + 1 == ck_next) {   // checkpoint ck_idx = H_{t+1} (ck_next lies past T without checkpoints)
+                    ck_next += p.C;
+                    ++ck_idx;
+                    if ((t + 1) < T) store_state(p.ckpt + ((size_t)bh * nck + ck_idx) * K * V);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(in_empty(s));
+                mbar_arrive(ypfull(c & 1));
             }
         }
         if (ok && p.HT != nullptr) store_state(p.HT + sbase);
