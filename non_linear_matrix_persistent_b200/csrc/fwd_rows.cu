@@ -146,7 +146,8 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
         // one chunk of TC steps per outer iteration: the ring and readout waits and
         // arrivals stay out of the step loop, whose body is then one straight
         // block (with the waits inside it, under a per-step test, the scan took
-        // 5.97 instead of 5.01 ms at the long B = 1 workload)
+        // 5.97 instead of 5.01 ms at the long B = 1 workload), unrolled by 4
+        // (5.01 -> 4.83 ms; by 8 or 16, 5.07 and 5.93 ms)
         for (int c = 0; c < nchunks && ok; ++c) {
             const int s = c % C::S, nt = min(C::TC, T - c * C::TC);
             const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
             if (ok && c >= 2)
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
             if (!ok) break;
+#pragma unroll 4
             for (int tt = 0; tt < nt; ++tt) {
                 const int t = c * C::TC + tt;
                 // both rows of h_{t-1} to every lane.  The buffer alternates by step:
