@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
         bool ok = true;
         // one chunk of TC steps per outer iteration: the ring and readout waits
         // and arrivals stay out of the step loop, whose body is one straight block
+        // (1.73 -> 1.57 ms at the 410M layer), unrolled by 2 (1.56 ms; by 4, 2.11)
         for (int c = 0; c < nchunks && ok; ++c) {
             const int s = c % C::S, nt = min(C::TC, T - c * C::TC);
             const uint8_t* st = smem + C::OFF_RING + s * C::STAGE_BYTES;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
             if (ok && c >= 2)
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(ypempty(c & 1), ((c >> 1) - 1) & 1, abort_flag, p));
             if (!ok) break;
+#pragma unroll 2
             for (int tt = 0; tt < nt; ++tt) {
                 const int t = c * C::TC + tt;
                 // H_{t-1} W: the state as compensated hi + lo bf16 A fragments
