@@ -159,44 +159,6 @@ __device__ __forceinline__ int ag_off(int m, int k) {
     return (k >> 3) * (128 * 16) + (m >> 3) * 128 + (k & 7) * 16 + (m & 7) * 2;
 }
 
-// The bf16 state values (round to nearest) of one thread's RT rows of its
-// column in a state operand, at the thread's own position tp within it:
-// tp = operand + (j/8)·(R·16) + (j%8)·16 + (nloc/8)·128 + (nloc%8)·2, the
-// layout of write_state_operand_hi<C, R> (the next 8-row group 128 bytes on).
-template <class C>
-__device__ __forceinline__ void put_state_hi(uint8_t* tp, const float (&h)[C::RT]) {
-    auto pack = [](float a, float b) {
-        const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-        return *reinterpret_cast<const uint32_t*>(&v);
-    };
-    if constexpr (C::RT % 8 == 0) {
-#pragma unroll
-        for (int g = 0; g < C::RT / 8; ++g)
-            *reinterpret_cast<uint4*>(tp + g * 128) =
-                make_uint4(pack(h[8 * g], h[8 * g + 1]), pack(h[8 * g + 2], h[8 * g + 3]),
-                           pack(h[8 * g + 4], h[8 * g + 5]), pack(h[8 * g + 6], h[8 * g + 7]));
-    } else {
-        *reinterpret_cast<uint2*>(tp) = make_uint2(pack(h[0], h[1]), pack(h[2], h[3]));
-    }
-}
-template <class C>
-__device__ __forceinline__ void get_state_hi(const uint8_t* tp, float (&h)[C::RT]) {
-    if constexpr (C::RT % 8 == 0) {
-#pragma unroll
-        for (int g = 0; g < C::RT / 8; ++g) {
-            const uint4 w = *reinterpret_cast<const uint4*>(tp + g * 128);
-            h[8 * g + 0] = bf16lo_to_f32(w.x); h[8 * g + 1] = bf16hi_to_f32(w.x);
-            h[8 * g + 2] = bf16lo_to_f32(w.y); h[8 * g + 3] = bf16hi_to_f32(w.y);
-            h[8 * g + 4] = bf16lo_to_f32(w.z); h[8 * g + 5] = bf16hi_to_f32(w.z);
-            h[8 * g + 6] = bf16lo_to_f32(w.w); h[8 * g + 7] = bf16hi_to_f32(w.w);
-        }
-    } else {
-        const uint2 w = *reinterpret_cast<const uint2*>(tp);
-        h[0] = bf16lo_to_f32(w.x); h[1] = bf16hi_to_f32(w.x);
-        h[2] = bf16lo_to_f32(w.y); h[3] = bf16hi_to_f32(w.y);
-    }
-}
-
 // Stores the extra output row (TMEM lane XLANE) of one tile, its R columns,
 // to dst[0 .. R).  Warp-collective over lane quarter 0; thread XLANE stores,
 // and only when `store` is set.

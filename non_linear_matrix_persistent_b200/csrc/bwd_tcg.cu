@@ -14,8 +14,10 @@
 // H_{c·C} with the forward's epilogue and the state as one bf16 operand (the
 // pages' backward recomputes states rather than storing them, §2.2; the
 // exact fp32 checkpoint every C <= 16 steps bounds that rounding), its states
-// and Z's go to a workspace
-// scratch, and the chunk is then walked in reverse; the recompute of one
+// and Z's stay on chip for V = 128 (in tensor memory and a ring of bf16
+// state operands, as in bwd_tc.cu: 32.7 -> 27.6 ms at the 7B-MoE training
+// shape with C = 8) or go to a workspace scratch for the other shapes, and
+// the chunk is then walked in reverse; the recompute of one
 // chunk and the reverse walk of the next run interleaved, each chain with its
 // own accumulators and MMA issuer.  Per step and tile three tcgen05 GEMMs:
 //   recompute      D = Wᵀ · H_{t-1}ᵀ   (M = MX state columns, N = the tile's rows, bf16 state)
@@ -46,10 +48,15 @@
 
 namespace m2rnn {
 
-template <int KS_, int V_>
+// OC: the recomputed chunk stays on chip (the Z's in tensor memory, the
+// states in a ring of bf16 operands, as in bwd_tc.cu); for V = 128 with a
+// checkpoint stride the tensor memory holds.  Otherwise the chunk goes
+// through a global-memory scratch.
+template <int KS_, int V_, bool OC_ = false>
 struct BwdTcgCfg {
     static constexpr int K = KS_;             // state rows of this CTA's slice
     static constexpr int V = V_;
+    static constexpr bool OC = OC_;
     static constexpr int MX = V <= 64 ? 64 : 128;   // M of every MMA; state columns j < V are real
     static constexpr int P = K >= 32 ? 2 : 1;       // row tiles with independent chains
     static constexpr int R = K / P;                 // rows per tile
@@ -62,7 +69,10 @@ struct BwdTcgCfg {
     static constexpr int NWE = P * WPT;             // epilogue warps
     static constexpr int NSLOT = P * SUBS;          // dv partials per (t, j)
     static constexpr int LG = MX == 64 ? 16 : 32;   // lanes that share a row block (one column each)
-    static constexpr int CMAX = 16;                 // max steps per checkpoint chunk
+    // on chip: per step one TMEM column per thread and row, NSLOT·RT columns a
+    // lane quarter, in the upper 256 columns
+    static constexpr int SCR_COL = 256, SCR_STEP = NSLOT * RT;
+    static constexpr int CMAX = OC ? (256 / SCR_STEP < 16 ? 256 / SCR_STEP : 16) : 16;   // max steps per chunk
     static constexpr int W_MREV = NWE, W_MREC = NWE + 1, W_STORE = NWE + 2, W_PROD = NWE + 3;
     static constexpr int NTHREADS = (NWE + 4) * 32;
     static constexpr int NSTAGE = 3;                // input chunks: recompute of i, reverse of i-1, prefetch of i+1
@@ -70,6 +80,7 @@ struct BwdTcgCfg {
     static constexpr int W_BYTES = MX * MX * 2;     // W, zero-padded to MX x MX
     static constexpr int B_BYTES = NT * V * 2;      // one state / dA operand (hi and lo)
     static constexpr int BS_BYTES = MX * R * 2;     // H_{t-1} hi operand of the dW MMA (MX rows)
+    static constexpr int NBR = CMAX + 2;            // on chip: state-operand ring slots (R rows each)
     static constexpr int ST_K = 0;                  // the slice's K values of k and q per step
     static constexpr int ST_Q = CMAX * K * 2;
     static constexpr int ST_V = 2 * CMAX * K * 2;
@@ -83,10 +94,13 @@ struct BwdTcgCfg {
     static constexpr int DQ_BYTES = CMAX * 4 * K * 4;            // [CMAX][4 quarters][K]
 
     static constexpr int OFF_W = 0;
-    static constexpr int OFF_BR = OFF_W + W_BYTES;               // recompute state operands per tile
-    static constexpr int OFF_BD = OFF_BR + P * B_BYTES;          // dA operands per tile
-    static constexpr int OFF_BS = OFF_BD + P * B_BYTES;          // H_{t-1} hi operands per tile
-    static constexpr int OFF_RING = (OFF_BS + P * BS_BYTES + 1023) / 1024 * 1024;
+    static constexpr int OFF_BD = OFF_W + W_BYTES;               // dA operands per tile
+    // recompute state operands per tile, then H_{t-1} hi operands per tile; on
+    // chip instead one ring [NBR][P] of BS_BYTES operands serving both
+    static constexpr int OFF_BR = OFF_BD + P * B_BYTES;
+    static constexpr int OFF_BS = OFF_BR + (OC ? 0 : P * B_BYTES);
+    static constexpr int BR_END = OC ? OFF_BR + NBR * P * BS_BYTES : OFF_BS + P * BS_BYTES;
+    static constexpr int OFF_RING = (BR_END + 1023) / 1024 * 1024;
     static constexpr int OFF_CK = OFF_RING + NSTAGE * STAGE_BYTES;   // the next checkpoint (fp32 [K][V])
     static constexpr int OFF_PART = OFF_CK + K * V * 4;
     static constexpr int FIXED = OFF_PART + 512;                 // + barriers and the TMEM slot
@@ -105,7 +119,7 @@ struct BwdTcgCfg {
     static constexpr int REV_COL = 0;                            // G-propagation accumulators, NT columns per tile
     static constexpr int REC_COL = P * NT;                       // recompute accumulators
     static constexpr int DW_COL = 2 * P * NT;                    // dW accumulator (V columns)
-    static constexpr int TMEM_COLS = (DW_COL + V <= 64) ? 64 : (DW_COL + V <= 128) ? 128
+    static constexpr int TMEM_COLS = OC ? 512 : (DW_COL + V <= 64) ? 64 : (DW_COL + V <= 128) ? 128
                                    : (DW_COL + V <= 256) ? 256 : 512;
 
     static_assert(K == 16 || K == 32 || (K == 64 && MX == 64), "slice rows");
@@ -115,6 +129,8 @@ struct BwdTcgCfg {
     static_assert((MX == 64 && V % 8 == 0) || (MX == 128 && V % 16 == 0), "N of the dW MMA");
     static_assert(NTHREADS <= 1024, "block size");
     static_assert(DW_COL + V <= TMEM_COLS && TMEM_COLS <= 512, "TMEM columns");
+    static_assert(!OC || (MX == 128 && DW_COL + V <= SCR_COL && CMAX * SCR_STEP <= 256 && CMAX >= 8),
+                  "on-chip chunk: 128-column states, scratch above the accumulators");
     static_assert(OFF_W % 1024 == 0 && OFF_BR % 128 == 0 && OFF_BD % 128 == 0 && OFF_BS % 128 == 0 &&
                   OFF_RING % 128 == 0 && OFF_CK % 128 == 0 && OFF_PART % 16 == 0 && OFF_DQ % 16 == 0 &&
                   OFF_BAR % 8 == 0, "alignment of shared-memory regions");
@@ -184,9 +200,9 @@ __device__ __forceinline__ float reduce_scatter(float* a, int lane, int& row) {
     }
 }
 
-template <int KS, int V>
-__global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_kernel(const Params p) {
-    using C = BwdTcgCfg<KS, V>;
+template <int KS, int V, bool OC>
+__global__ void __launch_bounds__(BwdTcgCfg<KS, V, OC>::NTHREADS, 1) m2rnn_bwd_tcg_kernel(const Params p) {
+    using C = BwdTcgCfg<KS, V, OC>;
     constexpr int K = C::K;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -266,9 +282,20 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
         const int row0 = tile * C::R + nloc;        // first slice row of this thread
         const int slot = tile * C::SUBS + sub;
         const size_t sbase = ((size_t)bh * KF + koff) * V;   // this slice's rows of dH_T / dH0
-        uint8_t* Br = smem + C::OFF_BR + tile * C::B_BYTES;
+        uint8_t* Br = smem + C::OFF_BR + tile * C::B_BYTES;     // (not on chip)
         uint8_t* Bd = smem + C::OFF_BD + tile * C::B_BYTES;
-        uint8_t* Bs = smem + C::OFF_BS + tile * C::BS_BYTES;
+        uint8_t* Bs = smem + C::OFF_BS + tile * C::BS_BYTES;    // (not on chip)
+        // On chip: the Z's of the chunk in TMEM (thread l of warp w in lane
+        // 32·(w mod 4) + l, columns SCR_COL + x·SCR_STEP + slot·RT + r for
+        // scratch slot x), the states H_{c0+u} in a ring of bf16 operands of
+        // R rows (this thread's values at brt, slot x at x·RING_STEP), which
+        // the recompute MMA of step c0+u and the dW MMA of the same step read,
+        // in the slot orders of bwd_tc.cu (scratch: u for even phases, CS-1-u
+        // for odd ones; ring: u and CS+1-u).
+        constexpr int RING_STEP = C::P * C::BS_BYTES;
+        const int tpos = (j >> 3) * (C::R * 16) + (j & 7) * 16 + (nloc >> 3) * 128 + (nloc & 7) * 2;
+        uint8_t* const brt = smem + C::OFF_BR + tile * C::BS_BYTES + tpos;
+        const uint32_t scr = tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)(C::SCR_COL + slot * C::RT);
         const uint32_t lanes = (uint32_t)(qd * 32) << 16;
         const uint32_t tb_rev = tmem + lanes + (uint32_t)(C::REV_COL + tile * C::NT + nsub);
         const uint32_t tb_rec = tmem + lanes + (uint32_t)(C::REC_COL + tile * C::NT + nsub);
@@ -324,6 +351,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
         };
 
         float G[C::RT], h[C::RT], zc[C::RT], hpc[C::RT];
+        uint32_t szr[C::RT];   // on chip: the Z's of the next reverse step as loaded from TMEM
 #pragma unroll
         for (int r = 0; r < C::RT; ++r)
             G[r] = (p.dHT != nullptr && jv) ? p.dHT[sbase + (size_t)(row0 + r) * V + j] : 0.f;
@@ -344,6 +372,24 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
             const uint8_t* stv = stage(m + C::NSTAGE - 1);
             const int pb = (m + C::NPART - 1) % C::NPART;   // partial-sum buffer of chunk m-1
             float* const part = reinterpret_cast<float*>(smem + C::OFF_PART + pb * C::PART_BYTES);
+            // on chip: slot walks of this phase's recompute and reverse chunks
+            const bool odd = (m & 1) != 0;
+            uint8_t* const rec_ring = brt + (odd ? (CS + 1) * RING_STEP : 0);
+            uint8_t* const rev_ring = brt + (odd ? 0 : (CS + 1) * RING_STEP);
+            const int rec_rstep = odd ? -RING_STEP : RING_STEP;
+            const uint32_t rec_scr = scr + (uint32_t)(odd ? (CS - 1) * C::SCR_STEP : 0);
+            const uint32_t rev_scr = scr + (uint32_t)(odd ? 0 : (CS - 1) * C::SCR_STEP);
+            const int rec_sstep = odd ? -C::SCR_STEP : C::SCR_STEP;
+            auto load_rev = [&](int u) {   // the reverse step of chunk step u: its Z's and H_{t-1}
+                if constexpr (C::OC) {
+                    tc_wait_st();
+                    tmem_ld_32x32b<C::RT>(rev_scr - (uint32_t)(u * rec_sstep), szr);
+                    get_state_hi<C>(rev_ring - u * rec_rstep, hpc);
+                } else {
+                    ld_vec(Sz, sslot(m - 1, u), zc);
+                    ld_vec(Sst, sslot(m - 1, u), hpc);
+                }
+            };
 
             if (has_rev) {
                 const int i = m - 1;
@@ -356,8 +402,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                     if (!ok) break;
                 }
                 // before the recompute below stores its first state (same slot)
-                ld_vec(Sz, sslot(m - 1, lenv - 1), zc);
-                ld_vec(Sst, sslot(m - 1, lenv - 1), hpc);
+                load_rev(lenv - 1);
             }
             if (has_rec) {
                 ok = __all_sync(0xffffffffu,
@@ -370,8 +415,12 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 for (int r = 0; r < C::RT; ++r) h[r] = jv ? ck[(row0 + r) * V + j] : 0.f;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(ck_empty);
-                st_vec(Sst, sslot(m, 0), h);
-                if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
+                if constexpr (C::OC) {
+                    put_state_hi<C>(rec_ring, h);
+                } else {
+                    st_vec(Sst, sslot(m, 0), h);
+                    if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rec(tile));
@@ -393,6 +442,13 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                     for (int r = 0; r < C::RT; ++r)
                         G[r] = fmaf(fprev, G[r], __uint_as_float(dhi[r]) + __uint_as_float(dlo[r]));
                     tc_fence_before();
+                } else if constexpr (C::OC) {
+                    tc_wait_ld();   // the chunk's first Z's
+                }
+                if constexpr (C::OC) {
+                    reg_fence(szr);
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r) zc[r] = __uint_as_float(szr[r]);
                 }
                 const float dyj = bf16_at(stv, C::ST_DY + (u + 1) * V * 2);
                 const float vj = bf16_at(stv, C::ST_V + u * V * 2);
@@ -413,15 +469,13 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 }
                 if (jv) {
                     write_state_operand<C, true>(Bd, dA, j, nloc);
-                    write_dw_a_operand<C>(Bs, hpc, j, nloc);   // the dW MMA reads the hi half only
+                    // the dW MMA reads H_{t-1} (hi half only): on chip, from the ring
+                    if constexpr (!C::OC) write_dw_a_operand<C>(Bs, hpc, j, nloc);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready_rev(tile));
-                if (u > 0) {
-                    ld_vec(Sz, sslot(m - 1, u - 1), zc);
-                    ld_vec(Sst, sslot(m - 1, u - 1), hpc);
-                }
+                if (u > 0) load_rev(u - 1);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) dfp += __shfl_xor_sync(0xffffffffu, dfp, o);
                 if (lane == 0) part[(C::DFP / 4) + u * C::NWE + warp] = dfp;
@@ -454,11 +508,19 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                     zz[r] = tanh_exp(a);
                     h[r] = fmaf(g, zz[r] - h[r], h[r]);
                 }
-                st_vec(Sz, sslot(m, u), zz);
-                if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
+                if constexpr (C::OC) {
+                    uint32_t zb[C::RT];
+#pragma unroll
+                    for (int r = 0; r < C::RT; ++r) zb[r] = __float_as_uint(zz[r]);
+                    tmem_st_32x32b<C::RT>(rec_scr + (uint32_t)(u * rec_sstep), zb);
+                } else {
+                    st_vec(Sz, sslot(m, u), zz);
+                    if (u + 1 < lenr) st_vec(Sst, sslot(m, u + 1), h);   // H_{c0+len} is not read back
+                }
                 tc_fence_before();
                 if (u + 1 < lenr) {
-                    if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
+                    if constexpr (C::OC) put_state_hi<C>(rec_ring + (u + 1) * rec_rstep, h);
+                    else if (jv) write_state_operand_hi<C>(Br, h, j, nloc);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bready_rec(tile));
@@ -472,6 +534,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 return true;
             };
             const int nsteps = max(lenr, lenv);
+#pragma unroll 2   // (32.2 -> 31.8 ms at the 7B-MoE training shape)
             for (int s = 0; s < nsteps && ok; ++s) {
                 if (s < lenv) ok = rev_step(s);
                 if (ok && s < lenr) ok = rec_step(s);
@@ -501,6 +564,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                 }
             }
         }
+        if constexpr (C::OC) tc_wait_st();   // no scratch store in flight when the columns are freed
         if (ok && jv) {
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) p.dH0[sbase + (size_t)(row0 + r) * V + j] = G[r];
@@ -594,7 +658,11 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                         }
                         ++nbr[tile];
                         tc_fence_after();
-                        const uint32_t bs = smem_u32(smem + C::OFF_BS + tile * C::BS_BYTES);
+                        // H_{t-1} of reverse step u: on chip, the ring slot of chunk step len-1-u
+                        const int us = len - 1 - u;
+                        const uint32_t bs = smem_u32(
+                            smem + (C::OC ? C::OFF_BR + (((i & 1) ? CS + 1 - us : us) * C::P + tile) * C::BS_BYTES
+                                          : C::OFF_BS + tile * C::BS_BYTES));
                         const uint32_t bd = smem_u32(smem + C::OFF_BD + tile * C::B_BYTES);
                         const uint32_t dt = tmem + (uint32_t)(C::REV_COL + tile * C::NT);
                         // G-propagation: A = W (MN-major view of the shared W buffer)
@@ -644,13 +712,17 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V>::NTHREADS, 1) m2rnn_bwd_tcg_k
                         }
                         ++nbr[tile];
                         tc_fence_after();
-                        const uint32_t br = smem_u32(smem + C::OFF_BR + tile * C::B_BYTES);
+                        // the state operand: on chip, the ring slot of chunk step u (R rows)
+                        constexpr int NB = C::OC ? C::R : C::NT;
+                        const uint32_t br = smem_u32(
+                            smem + (C::OC ? C::OFF_BR + (((i & 1) ? CS + 1 - u : u) * C::P + tile) * C::BS_BYTES
+                                          : C::OFF_BR + tile * C::B_BYTES));
                         const uint32_t dt = tmem + (uint32_t)(C::REC_COL + tile * C::NT);
                         // recompute: A = Wᵀ (K-major view of the shared W buffer)
 #pragma unroll
                         for (int ks = 0; ks < V / 16; ++ks)
                             tc_mma_f16_ss(dt, smem_desc(w0 + ks * 256, 128, C::MX * 16),
-                                          smem_desc(br + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_f,
+                                          smem_desc(br + ks * 2 * NB * 16, NB * 16, 128), idesc_f,
                                           ks > 0 ? 1u : 0u);
                         tc_commit(accfull_rec(tile));
                         issued[tile] = (int)(nbr[tile] - 1);
@@ -766,16 +838,23 @@ int tcg_slice_rows(int K, int V) {
     return K < cap ? K : cap;
 }
 
+// The chunk stays on chip for V = 128 when tensor memory holds C steps.
 template <int KS, int V>
+bool tcg_on_chip(int C) {
+    if constexpr (V == 128) return C <= BwdTcgCfg<KS, V, true>::CMAX;
+    return false;
+}
+
+template <int KS, int V, bool OC>
 cudaError_t launch_tcg(const Params& p0, cudaStream_t stream) {
-    using C = BwdTcgCfg<KS, V>;
+    using C = BwdTcgCfg<KS, V, OC>;
     Params p = p0;
     p.slices = p.K / KS;
     p.dw_parts = p.slices;   // one dW partial per slice
     const size_t ncta = (size_t)p.B * p.H * p.slices;
-    p.dv_part = p.scratch + 2 * (size_t)p.C * ncta * KS * C::MX;
+    p.dv_part = p.scratch + (OC ? 0 : 2 * (size_t)p.C * ncta * KS * C::MX);
     p.df_part = p.dv_part + (size_t)p.slices * p.B * p.H * p.T * V;
-    auto kern = m2rnn_bwd_tcg_kernel<KS, V>;
+    auto kern = m2rnn_bwd_tcg_kernel<KS, V, OC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)ncta, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
@@ -791,16 +870,28 @@ cudaError_t launch_tcg(const Params& p0, cudaStream_t stream) {
     return launch_dw_reduce(p, stream);
 }
 
+template <int KS, int V>
+cudaError_t launch_tcg_ks(const Params& p, cudaStream_t s) {
+    if constexpr (V == 128)
+        if (tcg_on_chip<KS, V>(p.C)) return launch_tcg<KS, V, true>(p, s);
+    return launch_tcg<KS, V, false>(p, s);
+}
+
 template <int V>
 cudaError_t launch_tcg_v(const Params& p, cudaStream_t s) {
     switch (tcg_slice_rows(p.K, V)) {
-        case 16: return launch_tcg<16, V>(p, s);
-        case 32: return launch_tcg<32, V>(p, s);
+        case 16: return launch_tcg_ks<16, V>(p, s);
+        case 32: return launch_tcg_ks<32, V>(p, s);
         case 64:
-            if constexpr (V <= 64) return launch_tcg<64, V>(p, s);
+            if constexpr (V <= 64) return launch_tcg_ks<64, V>(p, s);
             break;
     }
     return cudaErrorNotSupported;
+}
+
+bool tcg_chunk_on_chip(int K, int V, int C) {
+    if (V != 128) return false;
+    return tcg_slice_rows(K, V) == 16 ? tcg_on_chip<16, 128>(C) : tcg_on_chip<32, 128>(C);
 }
 
 }  // namespace
@@ -812,13 +903,13 @@ bool bwd_tcg_supported(int K, int V, int C) {
     return kv && C >= 1 && C <= BwdTcgCfg<16, 16>::CMAX;
 }
 
-// Per CTA: a dW partial and 2·C·KS·MX scratch values; with several slices per
-// pair, the slices' dv and df partials.
+// Per CTA: a dW partial and, unless the chunk stays on chip, 2·C·KS·MX
+// scratch values; with several slices per pair, the slices' dv and df partials.
 size_t bwd_tcg_workspace(int B, int H, int T, int K, int V, int C) {
     if (!bwd_tcg_supported(K, V, C)) return 0;
     const size_t ks = (size_t)tcg_slice_rows(K, V), nsl = (size_t)K / ks, mx = V <= 64 ? 64 : 128;
     const size_t ncta = (size_t)B * H * nsl;
-    size_t n = ncta * V * V + 2 * (size_t)C * ncta * ks * mx;
+    size_t n = ncta * V * V + (tcg_chunk_on_chip(K, V, C) ? 0 : 2 * (size_t)C * ncta * ks * mx);
     if (nsl > 1) n += nsl * (size_t)B * H * T * (V + 1);
     return sizeof(float) * n;
 }

@@ -70,7 +70,7 @@ WORKLOADS: Dict[str, Workload] = {
                                 backward=True),
     # the 7B-MoE layer shape trained: its inputs plus dY ~ N(0, 1)
     "layer7b_moe_train": Workload("layer7b_moe_train", B=4, H=32, T=4096, K=128, V=128,
-                                  gate_var=1.5, gate_shift=1.5, backward=True, ckpt_stride=16),
+                                  gate_var=1.5, gate_shift=1.5, backward=True),
 }
 
 

@@ -106,9 +106,10 @@ def test_tc_backward_every_shape_has_a_workspace(L):
     the extended-operand kernel's tensor-memory scratch (8 steps for K >= 64,
     16 for K = 32) needs only the dW partials (one per 64-row slice); longer
     strides there, and the other shapes, take the general-shape kernel, whose
-    workspace adds 2·C·KS·MX scratch values per CTA; K = 128 at V = 128 runs
-    four 32-row slices per pair, whose dv and df partials
-    (4·B·H·T·(V + 1) fp32) are summed after the kernel."""
+    workspace adds 2·C·KS·MX scratch values per CTA, except at V = 128 with a
+    stride its tensor memory holds (8 steps for 32-row slices, 16 for 16-row
+    ones); K = 128 at V = 128 runs four 32-row slices per pair, whose dv and
+    df partials (4·B·H·T·(V + 1) fp32) are summed after the kernel."""
     B, H, T, C = 2, 3, 5, 4
     for K in (16, 32, 64, 128):
         for V in (16, 32, 64, 128):
@@ -128,8 +129,13 @@ def test_tc_backward_every_shape_has_a_workspace(L):
     assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=64, V=64, C=12), 1) == pad(
         4 * (B * H * 64 * 64 + 2 * 12 * B * H * 64 * 64))
     ncta = B * H * 4
+    # V = 128 keeps a chunk of at most 8 steps (32-row slices) on chip: no scratch then
     assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=128, V=128, C=C), 1) == pad(
-        4 * (ncta * 128 * 128 + 2 * C * ncta * 32 * 128 + 4 * B * H * T * 129))
+        4 * (ncta * 128 * 128 + 4 * B * H * T * 129))
+    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=128, V=128, C=12), 1) == pad(
+        4 * (ncta * 128 * 128 + 2 * 12 * ncta * 32 * 128 + 4 * B * H * T * 129))
+    # 16-row slices (K = 16) hold 16 steps
+    assert L.m2rnn_workspace_size(_dims(B=B, H=H, T=T, K=16, V=128, C=16), 1) == pad(4 * B * H * 128 * 128)
 
 
 def test_fast_tanh_mode_workspace(L):

@@ -22,7 +22,7 @@ def test_per_step_counts_training_workload():
     f_only, _ = bench.per_step_counts(WORKLOADS["layer410m_fwd"])
     assert f_only["bytes"] == 2692 - 4 * K * V / 8   # no checkpoints without a backward
     _, bwd7 = bench.per_step_counts(WORKLOADS["layer7b_moe_train"])
-    assert bwd7["bytes"] == (4 * 128) * 2 + 4 + (3 * 128) * 4 + 4 + 4 * 128 * 128 / 16
+    assert bwd7["bytes"] == (4 * 128) * 2 + 4 + (3 * 128) * 4 + 4 + 4 * 128 * 128 / 8
 
 
 def test_kernel_digest_ignores_comments_only():

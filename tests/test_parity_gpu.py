@@ -454,7 +454,7 @@ def test_train_workload_sampled_head():
 
 def test_train_7b_moe_shape_sampled_head():
     """The 7B-MoE layer shape trained (B=4, H=32, K=V=128, T=4096; forward with
-    checkpoints every 16 steps, then the general-shape backward) in the
+    checkpoints every 8 steps, then the general-shape backward, chunk on chip) in the
     launch configuration the benchmark times; the oracle checks one whole head
     (all four batch rows, so dW[h] is complete), pair by pair."""
     w = WORKLOADS["layer7b_moe_train"]
