@@ -198,8 +198,9 @@ const char* m2rnn_status_string(m2rnn_status s);
 void m2rnn_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook: host-side fault injection for later launches (not part of the
- * method).  0 = none; 1 = the bf16 forward's input producer (tensor-core or
- * row kernel) stops after the first 16-step chunk, so the kernel's bounded
+ * method).  0 = none; 1 = the input producer of the bf16 forward (tensor-core
+ * or row kernel) and of the tensor-core backwards stops after its first chunk
+ * (16 steps forward, one checkpoint chunk backward), so the kernel's bounded
  * waits run out: the
  * call returns M2RNN_OK, the kernel exits early with undefined outputs and
  * m2rnn_get_device_status reports M2RNN_ERR_DEVICE_TIMEOUT (after about the

@@ -505,7 +505,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                 }
             }
         }
-        tc_wait_st();   // no scratch store may still be in flight when the columns are freed
+        tc_wait_st();   // no scratch store or load may still be in flight when the columns are freed
+        tc_wait_ld();
         if (ok) {
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) p.dH0[sbase + (size_t)(row0 + r) * V + j] = G[r];
@@ -551,6 +552,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         int last = -1, last_ck = -1;   // last chunk whose inputs / checkpoint were requested
         const int qkb = qk_pair(p, bh);   // k / q rows of this pair's head group
         for (int i = 0; i < nck; ++i) {
+            if (p.fault == 1 && i >= 1) break;   // injected: stop feeding the ring after the first chunk
             const int c0 = (nck - 1 - i) * CS, len = min(CS, T - c0), s = i % C::NSTAGE;
             if (i >= C::NSTAGE) {
                 const bool ok = __all_sync(
