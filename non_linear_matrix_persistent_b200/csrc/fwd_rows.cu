@@ -20,14 +20,16 @@
 // pairs, 64 of them, shared by the two rows) in four accumulator chains per
 // row; a lane's two adjacent columns move in 8-byte accesses.
 // Measured on B200 at the long B = 1 workload (1,024 rows on 128 SMs): one
-// row per warp 8.1 ms, two rows per warp (this kernel) 6.2 ms; slower were
-// the same with the h row stored as duplicated pairs (7.9 ms), a row pair
-// split over two warps by columns (8.5 ms) and a two-dimensional split of the
-// product over the lanes with a shuffle reduce-scatter (8.1 / 8.7 ms).
+// row per warp 8.1 ms, two rows per warp 6.2 ms (4.8 ms with the step loop
+// below); slower were the same with the h row stored as duplicated pairs
+// (7.9 ms), a row pair split over two warps by columns (8.5 ms) and a
+// two-dimensional split of the product over the lanes with a shuffle
+// reduce-scatter (8.1 / 8.7 ms).
 //
 // Arithmetic: fp32 products of the fp32 state with W (bf16 values, exact in
-// fp32), fp32 sums in a fixed order, the same exp-based tanh as the
-// tensor-core kernel (or tanh.approx.f32 in the fast-tanh mode), the blend
+// fp32), fp32 sums in a fixed order, the exp-based tanh of the tensor-core
+// kernels (here on packed pairs, tanh2_ex2, same bits; tanh.approx.f32 in the
+// fast-tanh mode), the blend
 // h + (1 - f)(z - h).  This is more precise than the tensor-core kernel's
 // compensated bf16 operand, so the two kernels' states agree to rounding, not
 // bit for bit; within this kernel a row's result does not depend on the rest
