@@ -92,8 +92,8 @@ struct BwdTcCfg {
     static constexpr int NWE = P * WPT;       // epilogue warps
     static constexpr int NSLOT = P * SUBS;    // dv partials per (t, j); also the epilogue warps per lane quarter
     // Recompute scratch in tensor memory: per step, one 32-bit column per
-    // state element (1 - Z² and Z - H_{t-1} as an fp16 pair), a lane quarter's
-    // NSLOT warps with RT columns each; SCR_COLS columns hold CMAX steps.
+    // state element (Z_t, fp32), a lane quarter's NSLOT warps with RT columns
+    // each; SCR_COLS columns hold CMAX steps.
     static constexpr int SCR_COL = 256, SCR_COLS = 256;
     static constexpr int SCR_STEP = NSLOT * RT;
     static constexpr int CMAX = SCR_COLS / SCR_STEP < 16 ? SCR_COLS / SCR_STEP : 16;   // max steps per chunk
@@ -286,12 +286,12 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
         // dA = (1-f) G (1 - Z²), which the carry G propagates, keeps the fp32 Z
         // (an fp16 (1 - Z², Z - H_{t-1}) pair in one column was measured: its
         // rounding, carried back through G, took the worst (b, h) pair's
-        // gradients from 6e-3 to 9e-3 of the oracle's).  One set of CMAX slots serves both chains: the
-        // chunk recomputed in phase i stores step u in slot u for even i and
-        // in slot C-1-u for odd i, so in phase i+1 the recompute writes exactly
-        // the slots the reverse walk (which reads its chunk from step len-1
-        // down, one step ahead) has already read.  Only the thread that wrote
-        // a value reads it back.
+        // gradients from 6e-3 to 9e-3 of the oracle's).  One set of CMAX slots
+        // serves both chains: the chunk recomputed in phase i stores step u in
+        // slot u for even i and in slot C-1-u for odd i, so in phase i+1 the
+        // recompute writes exactly the slots the reverse walk (which reads its
+        // chunk from step len-1 down, one step ahead) has already read.  Only
+        // the thread that wrote a value reads it back.
         const uint32_t scr = tmem + lanes + (uint32_t)(C::SCR_COL + slot * C::RT);
         // State operands H_{c0+u} (bf16, round to nearest) in a ring of CS + 2
         // slots per tile: the recompute MMA of step c0+u reads slot x(u), and
