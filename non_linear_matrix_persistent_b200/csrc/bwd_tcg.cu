@@ -1,6 +1,7 @@
-// M²RNN backward (BPTT) on the sm_100a tensor cores for every state shape the
-// V = 64 kernel of bwd_tc.cu does not take: V in {16, 32, 128}, and K = 16 at
-// any V.
+// M²RNN backward (BPTT) on the sm_100a tensor cores for every state shape and
+// checkpoint stride the V = 64 kernel of bwd_tc.cu does not take: V in
+// {16, 32, 128}, K = 16 at any V, and strides beyond that kernel's on-chip
+// chunk.
 //
 // The chain rule of the recurrence (gist.science technical summary of
 // "M²RNN: Non-Linear RNNs with Matrix-Valued States for Scalable Language
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V, OC>::NTHREADS, 1) m2rnn_bwd_t
         const uint32_t lanes = (uint32_t)(qd * 32) << 16;
         const uint32_t tb_rev = tmem + lanes + (uint32_t)(C::REV_COL + tile * C::NT + nsub);
         const uint32_t tb_rec = tmem + lanes + (uint32_t)(C::REC_COL + tile * C::NT + nsub);
-        // Scratch per CTA (layout of bwd_tc.cu): C slots of states H_{c0+u} and
+        // Global scratch per CTA (not on chip): C slots of states H_{c0+u} and
         // C slots of Z_{c0+u}; the chunk recomputed in phase i stores step u in
         // slot u for even i and C-1-u for odd i, so the next phase's recompute
         // overwrites only slots the reverse walk has read.  Slot x of CTA b is
