@@ -18,7 +18,9 @@ gate f_t in [0, 1]) have exact special cases that every kernel must reproduce:
 
 Every case runs in every forward mode (tensor-core, fast-tanh, register-
 resident mma.sync, fp32 debug) and in both backwards, against the fp64
-oracle at the tolerances of the other parity tests.  The last test checks
+oracle at the tolerances of the other parity tests.  One test holds every
+backward to exact power-of-two scaling of the incoming gradients (their
+magnitude is free, so the path must not depend on it), and the last checks
 the full-size training workload on several heads, pair by pair.
 """
 import json
@@ -76,6 +78,8 @@ def _edge_inputs(case, mode, K=64, V=64, T=24, B=2, H=3, seed=0, backward=False)
         x["f"] = torch.zeros_like(x["f"])
     elif case == "w0":
         x["W"] = torch.zeros_like(x["W"])
+    elif case == "drawn":
+        pass
     elif case == "sat":
         # powers of two keep the bf16 values exact.  k, v x64 make the rank-one
         # term dominate (|A| > 10 for over half of the elements, > 44 for over a
@@ -187,6 +191,33 @@ def test_edge_backward(case, mode, K, V):
         assert np.abs(gr["dH0"] - dH0c).max() <= 1e-10
         _, rel = _errs(g["dH0"], dH0c)
         assert rel <= tol
+
+
+@pytest.mark.parametrize("mode", ["bf16", "fp32"])
+@pytest.mark.parametrize("K,V", [(64, 64), (128, 128), (32, 16)])
+def test_backward_exact_under_gradient_scaling(mode, K, V):
+    """Given the forward states, every gradient is linear in the incoming ones
+    (dy_t, dH_T), and scaling by a power of two commutes with every rounding
+    step of floating point as long as nothing overflows or underflows.  So
+    dY, dH_T scaled by 2^-40 and 2^40 (about 1e-12 and 1e12, far outside the
+    range of a 16-bit float, and gradients of a loss averaged over many tokens
+    are small) must give exactly the scaled gradients in every backward."""
+    w, x = _edge_inputs("drawn", mode, K=K, V=V, T=29, seed=5 * K + V, backward=True)
+    xc = _cuda(x)
+    dHT = torch.randn(w.B, w.H, K, V, generator=torch.Generator().manual_seed(6)).cuda()
+    a = api()
+    C = 8
+    _, _, ck = a.forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True)
+    ref = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, xc["dY"], dHT, ckpt_stride=C)
+    for e in (-40, 40):
+        s = 2.0 ** e
+        dY = (xc["dY"].float() * s).to(xc["dY"].dtype)
+        assert torch.equal(dY.float() / s, xc["dY"].float())   # the scaled input is exact
+        g = a.backward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], ck, dY, dHT * s, ckpt_stride=C)
+        torch.cuda.synchronize()
+        assert a.device_status() == 0
+        for n in NAMES:
+            assert torch.equal(g[n] / s, ref[n]), (e, n, float((g[n] / s - ref[n]).abs().max()))
 
 
 def _spectral_radii(W):
