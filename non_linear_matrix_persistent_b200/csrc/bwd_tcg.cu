@@ -504,10 +504,13 @@ __global__ void __launch_bounds__(BwdTcgCfg<KS, V, OC>::NTHREADS, 1) m2rnn_bwd_t
                 reg_fence(ahi);
                 float zz[C::RT];
 #pragma unroll
-                for (int r = 0; r < C::RT; ++r) {
-                    const float a = fmaf(kk[r], vj, __uint_as_float(ahi[r]));
-                    zz[r] = tanh_exp(a);
-                    h[r] = fmaf(g, zz[r] - h[r], h[r]);
+                for (int r = 0; r < C::RT; r += 2) {
+                    const float2 z2 = tanh2_ex2(make_float2(fmaf(kk[r], vj, __uint_as_float(ahi[r])),
+                                                            fmaf(kk[r + 1], vj, __uint_as_float(ahi[r + 1]))));
+                    zz[r] = z2.x;
+                    zz[r + 1] = z2.y;
+                    h[r] = fmaf(g, z2.x - h[r], h[r]);
+                    h[r + 1] = fmaf(g, z2.y - h[r + 1], h[r + 1]);
                 }
                 if constexpr (C::OC) {
                     uint32_t zb[C::RT];

@@ -176,10 +176,11 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
                     const float v0 = bf16lo_to_f32(vv), v1 = bf16hi_to_f32(vv);
                     const float a0 = fmaf(k0, v0, acc[nt][0]), a1 = fmaf(k0, v1, acc[nt][1]);
                     const float a2 = fmaf(k1, v0, acc[nt][2]), a3 = fmaf(k1, v1, acc[nt][3]);
-                    h[nt][0] = fmaf(gt, tanh_exp(a0) - h[nt][0], h[nt][0]);
-                    h[nt][1] = fmaf(gt, tanh_exp(a1) - h[nt][1], h[nt][1]);
-                    h[nt][2] = fmaf(gt, tanh_exp(a2) - h[nt][2], h[nt][2]);
-                    h[nt][3] = fmaf(gt, tanh_exp(a3) - h[nt][3], h[nt][3]);
+                    const float2 z01 = tanh2_ex2(make_float2(a0, a1)), z23 = tanh2_ex2(make_float2(a2, a3));
+                    h[nt][0] = fmaf(gt, z01.x - h[nt][0], h[nt][0]);
+                    h[nt][1] = fmaf(gt, z01.y - h[nt][1], h[nt][1]);
+                    h[nt][2] = fmaf(gt, z23.x - h[nt][2], h[nt][2]);
+                    h[nt][3] = fmaf(gt, z23.y - h[nt][3], h[nt][3]);
                 }
                 // readout partial over this warp's 16 rows: per column, q_i0 H[i0] + q_i1 H[i1],
                 // then a reduce-scatter over the 8 lanes of a column group (lane bits 2-4)

@@ -252,16 +252,17 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
                 } else {
                     // element pairs in packed fp32 instructions (the same rn operations
                     // as scalar code): 1.733 -> 1.713 ms at K = V = 64 and 9.25 -> 8.81 ms
-                    // at K = V = 128 with the accurate tanh
+                    // at K = V = 128 with the accurate tanh; the accurate tanh itself on
+                    // pairs too (tanh2_ex2, the same bits as tanh_exp): 1.50 -> 1.43 ms
+                    // and 7.68 -> 7.25 ms
                     const float2 vj2 = make_float2(vj, vj), g2 = make_float2(g, g);
 #pragma unroll
                     for (int r = 0; r < C::CH; r += 2) {
                         float2 a2 = __fadd2_rn(make_float2(__uint_as_float(ahi[r]), __uint_as_float(ahi[r + 1])),
                                                make_float2(__uint_as_float(alo[r]), __uint_as_float(alo[r + 1])));
                         a2 = __ffma2_rn(make_float2(kk[r], kk[r + 1]), vj2, a2);
-                        const float z0 = FAST ? tanh_approx(a2.x) : tanh_exp(a2.x);
-                        const float z1 = FAST ? tanh_approx(a2.y) : tanh_exp(a2.y);
-                        const float2 d2 = __fadd2_rn(make_float2(z0, z1), make_float2(-h[c0 + r], -h[c0 + r + 1]));
+                        const float2 z2 = FAST ? make_float2(tanh_approx(a2.x), tanh_approx(a2.y)) : tanh2_ex2(a2);
+                        const float2 d2 = __fadd2_rn(z2, make_float2(-h[c0 + r], -h[c0 + r + 1]));
                         const float2 h2 = __ffma2_rn(g2, d2, make_float2(h[c0 + r], h[c0 + r + 1]));
                         h[c0 + r] = h2.x;
                         h[c0 + r + 1] = h2.y;
