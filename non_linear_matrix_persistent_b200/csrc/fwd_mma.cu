@@ -176,7 +176,9 @@ __global__ void __launch_bounds__(FwdMmaCfg<K>::NTHREADS, 1) m2rnn_fwd_mma_kerne
                     const float v0 = bf16lo_to_f32(vv), v1 = bf16hi_to_f32(vv);
                     const float a0 = fmaf(k0, v0, acc[nt][0]), a1 = fmaf(k0, v1, acc[nt][1]);
                     const float a2 = fmaf(k1, v0, acc[nt][2]), a3 = fmaf(k1, v1, acc[nt][3]);
-                    const float2 z01 = tanh2_ex2(make_float2(a0, a1)), z23 = tanh2_ex2(make_float2(a2, a3));
+                    // tanh accurate near zero in relative terms: this kernel also
+                    // writes checkpoints for the backward
+                    const float2 z01 = tanh2_acc(make_float2(a0, a1)), z23 = tanh2_acc(make_float2(a2, a3));
                     h[nt][0] = fmaf(gt, z01.x - h[nt][0], h[nt][0]);
                     h[nt][1] = fmaf(gt, z01.y - h[nt][1], h[nt][1]);
                     h[nt][2] = fmaf(gt, z23.x - h[nt][2], h[nt][2]);

@@ -28,8 +28,9 @@
 //
 // Arithmetic: fp32 products of the fp32 state with W (bf16 values, exact in
 // fp32), fp32 sums in a fixed order, the exp-based tanh of the tensor-core
-// kernels (here on packed pairs, tanh2_ex2, same bits; tanh.approx.f32 in the
-// fast-tanh mode), the blend
+// kernels (here on packed pairs, tanh2_ex2, same bits; in the instantiation
+// that writes the backward's checkpoints tanh2_acc, which keeps its relative
+// accuracy near zero; tanh.approx.f32 in the fast-tanh mode), the blend
 // h + (1 - f)(z - h).  This is more precise than the tensor-core kernel's
 // compensated bf16 operand, so the two kernels' states agree to rounding, not
 // bit for bit; within this kernel a row's result does not depend on the rest
@@ -199,8 +200,10 @@ __global__ void __launch_bounds__(FwdRowsCfg<RS>::NTHREADS, 1) m2rnn_fwd_rows_ke
                 A1 = __ffma2_rn(make_float2(k1, k1), v2, A1);
                 const float g = 1.f - *reinterpret_cast<const float*>(st + C::ST_F + tt * 4);
                 {
-                    const float2 z01 = FAST ? make_float2(tanh_approx(A0.x), tanh_approx(A0.y)) : tanh2_ex2(A0);
-                    const float2 z23 = FAST ? make_float2(tanh_approx(A1.x), tanh_approx(A1.y)) : tanh2_ex2(A1);
+                    const float2 z01 = FAST   ? make_float2(tanh_approx(A0.x), tanh_approx(A0.y))
+                                      : CKPT ? tanh2_acc(A0) : tanh2_ex2(A0);
+                    const float2 z23 = FAST   ? make_float2(tanh_approx(A1.x), tanh_approx(A1.y))
+                                      : CKPT ? tanh2_acc(A1) : tanh2_ex2(A1);
                     h0 = __ffma2_rn(make_float2(g, g), __fadd2_rn(z01, make_float2(-h0.x, -h0.y)), h0);
                     h1 = __ffma2_rn(make_float2(g, g), __fadd2_rn(z23, make_float2(-h1.x, -h1.y)), h1);
                 }

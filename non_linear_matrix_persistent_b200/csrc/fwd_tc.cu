@@ -58,9 +58,12 @@
 
 namespace m2rnn {
 
-template <int K_, int V_, bool FAST_ = false>
+// NSPLIT: bf16 terms of the state operand, 2 (hi + lo, ~2^-17 of each value)
+// or 3 (hi + mid + lo, ~2^-26), the latter for the instantiation that writes
+// the backward's checkpoints.
+template <int K_, int V_, bool FAST_ = false, int NSPLIT_ = 2>
 struct FwdTcCfg {
-    static constexpr int K = K_, V = V_;
+    static constexpr int K = K_, V = V_, NSPLIT = NSPLIT_;
     // row tiles with independent chains: 4 at K = V = 128 with the accurate
     // tanh, where the epilogue (32 rows per thread) and the MMA (N = 128 per
     // tile) are both long enough that two more chains in flight pay (8.86 ->
@@ -70,7 +73,7 @@ struct FwdTcCfg {
     static constexpr int P = (V == 128 && K == 128 && !FAST_) ? 4 : 2;
     static constexpr int MPAD = V <= 64 ? 64 : 128;
     static constexpr int R = K / P;                       // state rows per tile
-    static constexpr int NT = 2 * R;                      // MMA N per tile (hi rows, then lo rows)
+    static constexpr int NT = NSPLIT * R;                 // MMA N per tile (hi rows, [mid rows,] lo rows)
     // row groups per tile served by separate warps of the same lane quarter,
     // so that each thread handles at most 16 rows (measured on B200 at
     // K = V = 64: 1.85 -> 1.75 ms per 2048-step scan of 128 (b, h) pairs)
@@ -78,7 +81,8 @@ struct FwdTcCfg {
     static constexpr int WPT = 4 * SUBS;                  // epilogue warps per tile
     static constexpr int RT = (MPAD == 64) ? R / (2 * SUBS) : R / SUBS;  // rows per thread
     static constexpr int CH = RT < 16 ? RT : 16;          // rows per tensor-memory load
-    static constexpr int TC = 16;                         // steps per ring stage
+    // steps per ring stage (8 for the three-term operand at V = 128, for shared memory)
+    static constexpr int TC = (NSPLIT == 3 && V == 128) ? 8 : 16;
     static constexpr int S = 4;                           // ring stages
     static constexpr int NWE = P * WPT;                   // epilogue warps
     static constexpr int W_PROD = NWE, W_MMA = NWE + 1, W_STORE = NWE + 2;
@@ -101,15 +105,68 @@ struct FwdTcCfg {
     static constexpr int OFF_BAR = OFF_Y + 2 * YBUF_BYTES;
     static constexpr int NBAR = 2 * S + 2 * P + 4;
     static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16;
-    static constexpr int TMEM_COLS = (P * NT <= 32) ? 32 : (P * NT <= 64) ? 64 : (P * NT <= 128) ? 128 : 256;
+    static constexpr int TMEM_COLS = (P * NT <= 32) ? 32 : (P * NT <= 64) ? 64 : (P * NT <= 128) ? 128
+                                   : (P * NT <= 256) ? 256 : 512;
 
     static_assert(K % (2 * P) == 0 && RT >= 4 && RT % 4 == 0, "unsupported K");
     static_assert(NTHREADS <= 1024, "block size");
     static_assert((MPAD == 64 && NT % 8 == 0) || (MPAD == 128 && NT % 16 == 0), "bad MMA N");
-    static_assert(NT <= 256 && V % 16 == 0, "bad shape");
+    static_assert(NT <= 256 && V % 16 == 0 && P * NT <= 512, "bad shape");
     static_assert(RT % CH == 0, "chunking");
     static_assert(SMEM_BYTES <= 227 * 1024, "smem");
 };
+
+// Operand terms of an instantiation: three when it writes checkpoints and the
+// MMA shape allows N = 3R (M = 128 needs N % 16 == 0), else two.
+template <int K, int V, bool FAST, bool CKPT>
+__host__ __device__ constexpr int fwd_split() {
+    using C2 = FwdTcCfg<K, V, FAST, 2>;
+    return CKPT && (C2::MPAD == 64 || (3 * C2::R) % 16 == 0) ? 3 : 2;
+}
+
+// Three-term state operand: hi = RN(x), mid = RN(x - hi), lo = RN(x - hi - mid)
+// in bf16 (each residual exact in fp32), at rows n, R + n and 2R + n of the
+// layout of write_state_operand.
+template <class C>
+__device__ __forceinline__ void write_state_operand3(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
+    auto split3 = [](float a, float b, uint32_t& hi, uint32_t& md, uint32_t& lo) {
+        const __nv_bfloat162 hp = __floats2bfloat162_rn(a, b);
+        hi = *reinterpret_cast<const uint32_t*>(&hp);
+        const float a1 = a - bf16lo_to_f32(hi), b1 = b - bf16hi_to_f32(hi);
+        const __nv_bfloat162 mp = __floats2bfloat162_rn(a1, b1);
+        md = *reinterpret_cast<const uint32_t*>(&mp);
+        const __nv_bfloat162 lp = __floats2bfloat162_rn(a1 - bf16lo_to_f32(md), b1 - bf16hi_to_f32(md));
+        lo = *reinterpret_cast<const uint32_t*>(&lp);
+    };
+    uint8_t* colbase = Bt + (j >> 3) * (C::NT * 16) + (j & 7) * 16;
+    if constexpr (C::RT % 8 == 0) {
+#pragma unroll
+        for (int g = 0; g < C::RT / 8; ++g) {
+            uint4 hi, md, lo;
+            split3(h[8 * g + 0], h[8 * g + 1], hi.x, md.x, lo.x);
+            split3(h[8 * g + 2], h[8 * g + 3], hi.y, md.y, lo.y);
+            split3(h[8 * g + 4], h[8 * g + 5], hi.z, md.z, lo.z);
+            split3(h[8 * g + 6], h[8 * g + 7], hi.w, md.w, lo.w);
+            const int n = nloc + 8 * g;
+            *reinterpret_cast<uint4*>(colbase + (n >> 3) * 128) = hi;
+            *reinterpret_cast<uint4*>(colbase + ((C::R + n) >> 3) * 128) = md;
+            *reinterpret_cast<uint4*>(colbase + ((2 * C::R + n) >> 3) * 128) = lo;
+        }
+    } else {
+        uint2 hi, md, lo;
+        split3(h[0], h[1], hi.x, md.x, lo.x);
+        split3(h[2], h[3], hi.y, md.y, lo.y);
+        const int n = nloc;
+        *reinterpret_cast<uint2*>(colbase + (n >> 3) * 128 + (n & 7) * 2) = hi;
+        *reinterpret_cast<uint2*>(colbase + ((C::R + n) >> 3) * 128 + ((C::R + n) & 7) * 2) = md;
+        *reinterpret_cast<uint2*>(colbase + ((2 * C::R + n) >> 3) * 128 + ((2 * C::R + n) & 7) * 2) = lo;
+    }
+}
+template <class C>
+__device__ __forceinline__ void write_operand(uint8_t* Bt, const float (&h)[C::RT], int j, int nloc) {
+    if constexpr (C::NSPLIT == 3) write_state_operand3<C>(Bt, h, j, nloc);
+    else write_state_operand<C>(Bt, h, j, nloc);
+}
 
 // FAST: tanh.approx.f32 (one SFU operation, ~2^-11 relative error) instead
 // of the exp-based formula; forward-only inference mode.  CKPT: the
@@ -121,7 +178,7 @@ struct FwdTcCfg {
 // measured slower at V = 128 (8.83 -> 9.15 ms) and equal at V = 64.
 template <int K, int V, bool FAST, bool CKPT>
 __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_tc_kernel(const Params p) {
-    using C = FwdTcCfg<K, V, FAST>;
+    using C = FwdTcCfg<K, V, FAST, fwd_split<K, V, FAST, CKPT>()>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // One CTA per (b, h) and slice of K rows (p.slices slices of the p.K state
@@ -203,7 +260,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
 #pragma unroll
             for (int r = 0; r < C::RT; ++r) ck[(size_t)(row0 + r) * V + j] = h[r];
         }
-        if (jv) write_state_operand<C>(Bt, h, j, nloc);
+        if (jv) write_operand<C>(Bt, h, j, nloc);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bready(tile));
@@ -224,20 +281,29 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
             const uint16_t* kt = reinterpret_cast<const uint16_t*>(st + C::ST_K + tt * K * 2) + row0;
 #pragma unroll
             for (int c0 = 0; c0 < C::RT; c0 += C::CH) {
-                uint32_t ahi[C::CH], alo[C::CH];
+                uint32_t ahi[C::CH], alo[C::CH], amd[C::CH];
                 if constexpr (C::MPAD == 64) {
                     // the two half-warps own rows [0, RT) and [RT, 2RT) of the warp's block
                     tmem_ld_16x32bx2<C::CH, C::RT>(tbase + c0, ahi);
-                    tmem_ld_16x32bx2<C::CH, C::RT>(tbase + C::R + c0, alo);
+                    tmem_ld_16x32bx2<C::CH, C::RT>(tbase + (C::NSPLIT - 1) * C::R + c0, alo);
+                    if constexpr (C::NSPLIT == 3) tmem_ld_16x32bx2<C::CH, C::RT>(tbase + C::R + c0, amd);
                 } else {
                     tmem_ld_32x32b<C::CH>(tbase + c0, ahi);
-                    tmem_ld_32x32b<C::CH>(tbase + C::R + c0, alo);
+                    tmem_ld_32x32b<C::CH>(tbase + (C::NSPLIT - 1) * C::R + c0, alo);
+                    if constexpr (C::NSPLIT == 3) tmem_ld_32x32b<C::CH>(tbase + C::R + c0, amd);
                 }
                 float kk[C::CH];
                 lds_bf16<C::CH>(kt + c0, kk);
                 tc_wait_ld();
                 reg_fence(ahi);
                 reg_fence(alo);
+                if constexpr (C::NSPLIT == 3) {
+                    // the mid and lo products first, then the hi product
+                    reg_fence(amd);
+#pragma unroll
+                    for (int r = 0; r < C::CH; ++r)
+                        alo[r] = __float_as_uint(__uint_as_float(amd[r]) + __uint_as_float(alo[r]));
+                }
                 if constexpr (FAST && C::MPAD == 128) {
                     // scalar: with the single-SFU tanh at V = 128 the packed form
                     // below measured 6% slower (6.07 -> 6.43 ms at B = 4, 32 heads,
@@ -254,14 +320,21 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
                     // as scalar code): 1.733 -> 1.713 ms at K = V = 64 and 9.25 -> 8.81 ms
                     // at K = V = 128 with the accurate tanh; the accurate tanh itself on
                     // pairs too (tanh2_ex2, the same bits as tanh_exp): 1.50 -> 1.43 ms
-                    // and 7.68 -> 7.25 ms
+                    // and 7.68 -> 7.25 ms.  The instantiation that writes the
+                    // backward's checkpoints takes tanh2_acc (the Taylor series below
+                    // |x| = 1/8): the exp form's absolute error of ~2e-7 is a large
+                    // relative error on small states, which heads whose recurrence
+                    // amplifies perturbations carry into the gradients (the 7B-MoE
+                    // shape's head 25: 4.1e-2 relative against 3.3e-3; 1.48 -> 1.52 ms
+                    // at the 410M training workload)
                     const float2 vj2 = make_float2(vj, vj), g2 = make_float2(g, g);
 #pragma unroll
                     for (int r = 0; r < C::CH; r += 2) {
                         float2 a2 = __fadd2_rn(make_float2(__uint_as_float(ahi[r]), __uint_as_float(ahi[r + 1])),
                                                make_float2(__uint_as_float(alo[r]), __uint_as_float(alo[r + 1])));
                         a2 = __ffma2_rn(make_float2(kk[r], kk[r + 1]), vj2, a2);
-                        const float2 z2 = FAST ? make_float2(tanh_approx(a2.x), tanh_approx(a2.y)) : tanh2_ex2(a2);
+                        const float2 z2 = FAST   ? make_float2(tanh_approx(a2.x), tanh_approx(a2.y))
+                                         : CKPT ? tanh2_acc(a2) : tanh2_ex2(a2);
                         const float2 d2 = __fadd2_rn(z2, make_float2(-h[c0 + r], -h[c0 + r + 1]));
                         const float2 h2 = __ffma2_rn(g2, d2, make_float2(h[c0 + r], h[c0 + r + 1]));
                         h[c0 + r] = h2.x;
@@ -271,7 +344,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
             }
             tc_fence_before();
             if (t + 1 < T) {
-                if (jv) write_state_operand<C>(Bt, h, j, nloc);
+                if (jv) write_operand<C>(Bt, h, j, nloc);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bready(tile));
@@ -467,7 +540,7 @@ __global__ void __launch_bounds__(FwdTcCfg<K, V, FAST>::NTHREADS, 1) m2rnn_fwd_t
 
 template <int K, int V, bool FAST, bool CKPT>
 static cudaError_t launch_fwd_tc_one(const Params& p, cudaStream_t stream) {
-    using C = FwdTcCfg<K, V, FAST>;
+    using C = FwdTcCfg<K, V, FAST, fwd_split<K, V, FAST, CKPT>()>;
     auto kern = m2rnn_fwd_tc_kernel<K, V, FAST, CKPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;

@@ -290,6 +290,22 @@ __device__ __forceinline__ float2 tanh2_ex2(float2 x) {
     const float2 d = __fadd2_rn(make_float2(ex2_approx(y.x), ex2_approx(y.y)), make_float2(1.f, 1.f));
     return __ffma2_rn(make_float2(-2.f, -2.f), make_float2(rcp_approx(d.x), rcp_approx(d.y)), make_float2(1.f, 1.f));
 }
+// tanh of two values with a small relative error at every argument.  The
+// exp form above loses relative accuracy near zero (1 - 2/(1 + e^{2x}) cancels
+// to an absolute error of ~2e-7, i.e. 1e-4 of the value at |x| = 1e-3); for
+// |x| < 1/8 this takes the odd Taylor series of tanh instead,
+//   x - x^3/3 + 2x^5/15 - 17x^7/315,
+// whose next term, 62x^9/2835, is below 2e-10 of x there (about one ulp in
+// fp32 with the rounding of the evaluation), and the exp form elsewhere
+// (relative error at most ~1.6e-6, at |x| = 1/8).
+__device__ __forceinline__ float2 tanh2_acc(float2 x) {
+    const float2 big = tanh2_ex2(x);
+    const float2 s = __fmul2_rn(x, x);
+    float2 q = __ffma2_rn(make_float2(-17.f / 315.f, -17.f / 315.f), s, make_float2(2.f / 15.f, 2.f / 15.f));
+    q = __ffma2_rn(q, s, make_float2(-1.f / 3.f, -1.f / 3.f));
+    const float2 small = __ffma2_rn(__fmul2_rn(x, s), q, x);
+    return make_float2(fabsf(x.x) < 0.125f ? small.x : big.x, fabsf(x.y) < 0.125f ? small.y : big.y);
+}
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

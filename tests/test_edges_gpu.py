@@ -18,10 +18,12 @@ gate f_t in [0, 1]) have exact special cases that every kernel must reproduce:
 
 Every case runs in every forward mode (tensor-core, fast-tanh, register-
 resident mma.sync, fp32 debug) and in both backwards, against the fp64
-oracle at the tolerances of the other parity tests.  One test holds every
-backward to exact power-of-two scaling of the incoming gradients (their
-magnitude is free, so the path must not depend on it), and the last checks
-the full-size training workload on several heads, pair by pair.
+oracle at the tolerances of the other parity tests.  One test holds the
+checkpointing forwards' states to a small relative error near zero (the
+gradients of heads whose recurrence amplifies perturbations depend on it), one
+holds every backward to exact power-of-two scaling of the incoming gradients
+(their magnitude is free, so the path must not depend on it), and the last
+checks the full-size training workload on several heads, pair by pair.
 """
 import json
 import os
@@ -191,6 +193,52 @@ def test_edge_backward(case, mode, K, V):
         assert np.abs(gr["dH0"] - dH0c).max() <= 1e-10
         _, rel = _errs(g["dH0"], dH0c)
         assert rel <= tol
+
+
+@pytest.mark.parametrize("B,H,K,V,mma", [(8, 16, 64, 64, False), (1, 2, 64, 64, False), (2, 2, 128, 128, False),
+                                         (2, 2, 64, 64, True)])
+def test_checkpoint_states_relative_accuracy_near_zero(B, H, K, V, mma):
+    """The forward that writes the backward's checkpoints (tensor-core kernel at
+    V = 64 and 128, row kernel for few pairs, mma.sync kernel) evaluates tanh
+    with a small relative error at every argument: gradients of heads whose
+    recurrence amplifies perturbations depend on the small states' relative
+    accuracy.  With W = 0, f = 0 and k_t = 0 except at the step before each
+    checkpoint, every state is 0 except the checkpointed one, which is then
+    tanh(k_t v_tᵀ) exactly (the product of two bf16 values is exact in fp32, and
+    the blend of a zero state adds nothing); k, v scaled by 2 put a third or
+    more of those pre-activations below 1e-2, where a tanh with the absolute
+    error of an exp-based form (~2e-7) would be off by 2e-5 or more of the
+    value, and some above 1/8, where the exp form is kept (relative error up
+    to ~1.6e-6 at 1/8)."""
+    w = Workload("rel0", B=B, H=H, T=33, K=K, V=V, seed=K + V + B)
+    x = make_inputs(w)
+    C = 8
+    x["W"] = torch.zeros_like(x["W"])
+    x["f"] = torch.zeros_like(x["f"])
+    for n in ("k", "v"):
+        x[n] = (x[n].float() * 2.0).to(x[n].dtype)
+    keep = torch.zeros(w.T, dtype=torch.bool)
+    keep[C - 1::C] = True
+    x["k"] = torch.where(keep[None, None, :, None], x["k"], torch.zeros_like(x["k"]))
+    xc = _cuda(x)
+    _, _, ck = api().forward(xc["k"], xc["v"], xc["q"], xc["f"], xc["W"], xc["H0"], ckpt_stride=C, want_ckpt=True,
+                             mma_sync=mma)
+    torch.cuda.synchronize()
+    assert api().device_status() == 0
+    k, v = x["k"].double().numpy(), x["v"].double().numpy()
+    for c in range(1, ck.shape[2]):
+        a = k[:, :, c * C - 1, :, None] * v[:, :, c * C - 1, None, :]
+        z = np.tanh(a)
+        got = ck[:, :, c].double().cpu().numpy()
+        assert np.all((got == 0) == (z == 0))
+        nz = z != 0
+        rel = np.abs(got[nz] - z[nz]) / np.abs(z[nz])
+        small = np.abs(a[nz]) < 0.125
+        assert small.mean() > 0.8 and (np.abs(a) < 1e-2).mean() > 0.25 and not small.all()   # the premise
+        _log("ckpt_rel_near_zero_B%d_H%d_K%d_V%d_mma%d" % (B, H, K, V, mma), c=c,
+             rel_small=float(rel[small].max()), rel_large=float(rel[~small].max()))
+        assert rel[small].max() <= 4e-7, (c, float(rel[small].max()))
+        assert rel[~small].max() <= 3e-6, (c, float(rel[~small].max()))
 
 
 @pytest.mark.parametrize("mode", ["bf16", "fp32"])
