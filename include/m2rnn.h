@@ -67,7 +67,13 @@ typedef enum {
     /* bf16 k/v/q/W inputs; the per-step H_{t-1}·W runs on the tcgen05 tensor
      * cores (bf16 operands, fp32 accumulation in tensor memory).  The fp32
      * state is fed to the MMA as a compensated pair of bf16 operands
-     * (hi + lo), so the operand carries about 16 bits of mantissa. */
+     * (hi + lo), so the operand carries about 16 bits of mantissa; a
+     * forward that writes checkpoints (ckpt != NULL) feeds it as three bf16
+     * terms (about 24 bits) and evaluates tanh with a small relative error
+     * near zero as well, since the backward's gradients can amplify the
+     * checkpoints' relative error (heads whose W has a spectral radius above
+     * 1).  y and H_T of the two kinds of call therefore agree to rounding,
+     * not bit for bit. */
     M2RNN_MODE_BF16_TC = 0,
     /* fp32 everything, CUDA-core FFMA and accurate tanhf: a slow reference
      * mode on the device. */
@@ -82,8 +88,9 @@ typedef enum {
     /* bf16 inputs, forward only, V = 64 and K in {16, 32, 64} (other shapes
      * return M2RNN_ERR_UNSUPPORTED_SHAPE): a latency-oriented alternative
      * forward with the state resident in registers (warp-level mma.sync, 16
-     * rows per warp, no per-step barrier).  Same compensated operand and
-     * accurate tanh as M2RNN_MODE_BF16_TC; its checkpoints may be passed to
+     * rows per warp, no per-step barrier).  Same compensated pair as
+     * M2RNN_MODE_BF16_TC, with the tanh that is accurate near zero in
+     * relative terms; its checkpoints may be passed to
      * m2rnn_backward in M2RNN_MODE_BF16_TC.  m2rnn_backward rejects this mode
      * (M2RNN_ERR_INVALID_ARG). */
     M2RNN_MODE_BF16_MMA_SYNC = 3
