@@ -13,7 +13,8 @@
 // here each chunk of C steps is recomputed from the forward's checkpoint
 // H_{c·C} with the forward kernel's epilogue, but with the state entering the
 // recompute product as one bf16 operand (round to nearest) rather than the
-// forward's compensated hi + lo pair: each chunk restarts from an exact fp32
+// forward's compensated operand (two or three bf16 terms): each chunk restarts
+// from an exact fp32
 // checkpoint, so the rounding cannot accumulate beyond C steps, and on three
 // full heads of the 410M training workload every (b, h) pair's gradients
 // stayed as close to the fp64 oracle as with the pair (worst dW 6.0e-3
@@ -39,9 +40,12 @@
 // otherwise take cross-lane shuffles:
 //   recompute:      Σ_l dy_{t-1}[l] H_{t-1}[i, l] = dq_{t-1}[i]
 //   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
-// The G-propagation MMA takes dA as a compensated pair (hi, then lo rows of
-// its operand) and sums both halves in one accumulator, two MMA groups of
-// N = R.  Software pipelining: the recompute of one chunk and the reverse
+// The G-propagation and dW MMAs take dA as one bf16 operand rounded to
+// nearest (N = R): with checkpoints from the forward's three-term state
+// operand, the worst (b, h) pair of three heads of the 410M training workload
+// stays at 5.7e-3 of the oracle (2.1e-3 with a compensated hi + lo pair, whose
+// second MMA group cost 0.17 ms: 3.11 -> 2.94 ms without it; with the older
+// two-term checkpoints the single operand had reached 1.2e-2).  Software pipelining: the recompute of one chunk and the reverse
 // walk of the chunk after it (in time) are independent chains, so the
 // epilogue interleaves them step for step, each with its own TMEM
 // accumulators and MMA issuer warp, sharing the scratch; each chain's MMA
@@ -85,7 +89,7 @@ struct BwdTcCfg {
     static constexpr int MX = 128;            // M of the recompute and G-propagation MMAs
     static constexpr int XLANE = 16;          // TMEM lane (and Ã row) of the extra output
     static constexpr int R = K / P;           // rows per tile
-    static constexpr int NT = 2 * R;          // G-propagation MMA N per tile (dA hi rows, then lo rows)
+    static constexpr int NT = R;              // dA operand rows per tile (the G-propagation MMA's N)
     // 8 rows per epilogue thread: two warps per TMEM lane quarter and tile at
     // R = 32 (each owning half of the tile's rows), one at R = 16.  Measured at
     // the training workload's shape: 16 rows per thread at R = 32 took 3.22
@@ -108,7 +112,7 @@ struct BwdTcCfg {
     static constexpr int NSTAGE = 3;          // input chunks: recompute of i, reverse of i-1, prefetch of i+1
 
     static constexpr int AX_BYTES = MX * V * 2;            // one extended A operand
-    static constexpr int B_BYTES = NT * V * 2;             // one tile's dA operand (hi + lo)
+    static constexpr int B_BYTES = NT * V * 2;             // one tile's dA operand (bf16)
     static constexpr int BR_BYTES = R * V * 2;             // one tile's state operand (bf16, R rows)
     static constexpr int NBR = CMAX + 2;                   // state-operand ring slots (see the epilogue)
     static constexpr int ST_K = 0;
@@ -422,7 +426,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                     dfp = fmaf(G[r], dz[r], dfp);
                     dvp = fmaf(dA[r], kk[r], dvp);
                 }
-                write_state_operand<C, true>(Bd, dA, j, nloc);
+                write_state_operand_hi<C>(Bd, dA, j, nloc);
                 if (xwriter) *xg = vbits;
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -544,8 +548,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                     tc_fence_after();
                     const uint32_t tcol = tmem + (uint32_t)((xd ? C::REV_COL : C::REC_COL) + tile * C::R);
                     float* dst = out + ((size_t)bh * T + max(t, 0)) * KF + koff + tile * C::R;
-                    // (both accumulators are R columns: the G-propagation sums dA's hi and
-                    // lo halves in the MMA, and the recompute's state operand has no lo half)
+                    // (both accumulators are R columns: dA and the recompute's state
+                    // operand are single bf16 operands)
                     store_xrow<C>(tcol, dst, lane == C::XLANE && t >= 0);
                     tc_fence_before();
                     __syncwarp();
@@ -608,7 +612,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
     } else if (warp == C::W_MREV) {
         // ------------------------------------------------------------ MMA issuer: reverse chain
         if (lane == 0) {
-            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::R, 1, 1);   // dA hi, then dA lo, one accumulator
+            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::R, 1, 1);   // dA (bf16)
             constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
             uint32_t nbr[C::P];
             int issued[C::P];
@@ -642,11 +646,6 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                             tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
                                           smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
                                           ks > 0 ? 1u : 0u);
-#pragma unroll
-                        for (int ks = 0; ks < V / 16; ++ks)   // lo rows R .. 2R-1 of the dA operand
-                            tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
-                                          smem_desc(bd + (C::R / 8) * 128 + ks * 2 * C::NT * 16, C::NT * 16, 128),
-                                          idesc_g, 1u);
 #pragma unroll
                         for (int ks = 0; ks < C::R / 16; ++ks)
                             tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::R * 16),
