@@ -40,8 +40,9 @@
 // otherwise take cross-lane shuffles:
 //   recompute:      Σ_l dy_{t-1}[l] H_{t-1}[i, l] = dq_{t-1}[i]
 //   G-propagation:  Σ_j v_t[j] dA_t[i, j]         = dk_t[i].
-// The G-propagation and dW MMAs take dA as one bf16 operand rounded to
-// nearest (N = R): with checkpoints from the forward's three-term state
+// For T <= 2048 the G-propagation and dW MMAs take dA as one bf16 operand
+// rounded to nearest (N = R; longer sequences keep the compensated pair, see
+// launch_bwd_tc_k): with checkpoints from the forward's three-term state
 // operand, the worst (b, h) pair of three heads of the 410M training workload
 // stays at 5.7e-3 of the oracle (2.1e-3 with a compensated hi + lo pair, whose
 // second MMA group cost 0.17 ms: 3.11 -> 2.94 ms without it; with the older
@@ -80,8 +81,11 @@ namespace m2rnn {
 // K state rows are handled as NSL independent slices of KS rows, one CTA
 // per (b, h, slice): the rows of H evolve independently given W, v_t and f_t,
 // so a slice needs only its own rows of k, q, the checkpoints and dH_T.
-template <int KS_, int NSL_>
+// PAIR: dA enters the G-propagation as a compensated hi + lo pair (two MMA
+// groups of N = R into one accumulator) instead of one bf16 operand.
+template <int KS_, int NSL_, bool PAIR_ = false>
 struct BwdTcCfg {
+    static constexpr bool PAIR = PAIR_;
     static constexpr int K = KS_;             // rows of this CTA's slice
     static constexpr int NSL = NSL_, KF = K * NSL, V = 64;
     static constexpr int P = 2;
@@ -89,7 +93,7 @@ struct BwdTcCfg {
     static constexpr int MX = 128;            // M of the recompute and G-propagation MMAs
     static constexpr int XLANE = 16;          // TMEM lane (and Ã row) of the extra output
     static constexpr int R = K / P;           // rows per tile
-    static constexpr int NT = R;              // dA operand rows per tile (the G-propagation MMA's N)
+    static constexpr int NT = PAIR ? 2 * R : R;   // dA operand rows per tile (hi rows, then lo rows with PAIR)
     // 8 rows per epilogue thread: two warps per TMEM lane quarter and tile at
     // R = 32 (each owning half of the tile's rows), one at R = 16.  Measured at
     // the training workload's shape: 16 rows per thread at R = 32 took 3.22
@@ -112,7 +116,7 @@ struct BwdTcCfg {
     static constexpr int NSTAGE = 3;          // input chunks: recompute of i, reverse of i-1, prefetch of i+1
 
     static constexpr int AX_BYTES = MX * V * 2;            // one extended A operand
-    static constexpr int B_BYTES = NT * V * 2;             // one tile's dA operand (bf16)
+    static constexpr int B_BYTES = NT * V * 2;             // one tile's dA operand (bf16, or hi + lo)
     static constexpr int BR_BYTES = R * V * 2;             // one tile's state operand (bf16, R rows)
     static constexpr int NBR = CMAX + 2;                   // state-operand ring slots (see the epilogue)
     static constexpr int ST_K = 0;
@@ -189,9 +193,9 @@ __device__ __forceinline__ void store_xrow(uint32_t tcol, float* dst, bool store
     }
 }
 
-template <int KS, int NSL>
+template <int KS, int NSL, bool PAIR>
 __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_kernel(const Params p) {
-    using C = BwdTcCfg<KS, NSL>;
+    using C = BwdTcCfg<KS, NSL, PAIR>;
     constexpr int K = C::K, KF = C::KF, V = C::V;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -426,7 +430,8 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                     dfp = fmaf(G[r], dz[r], dfp);
                     dvp = fmaf(dA[r], kk[r], dvp);
                 }
-                write_state_operand_hi<C>(Bd, dA, j, nloc);
+                if constexpr (C::PAIR) write_state_operand<C, true>(Bd, dA, j, nloc);
+                else write_state_operand_hi<C>(Bd, dA, j, nloc);
                 if (xwriter) *xg = vbits;
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
     } else if (warp == C::W_MREV) {
         // ------------------------------------------------------------ MMA issuer: reverse chain
         if (lane == 0) {
-            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::R, 1, 1);   // dA (bf16)
+            constexpr uint32_t idesc_g = idesc_bf16_f32(C::MX, C::R, 1, 1);   // dA (hi, then lo with PAIR)
             constexpr uint32_t idesc_w = idesc_bf16_f32(C::MPAD, V, 0, 0);
             uint32_t nbr[C::P];
             int issued[C::P];
@@ -646,6 +651,13 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
                             tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
                                           smem_desc(bd + ks * 2 * C::NT * 16, C::NT * 16, 128), idesc_g,
                                           ks > 0 ? 1u : 0u);
+                        if constexpr (C::PAIR) {
+#pragma unroll
+                            for (int ks = 0; ks < V / 16; ++ks)   // lo rows R .. 2R-1 of the dA operand
+                                tc_mma_f16_ss(dt, smem_desc(ag + ks * 2 * C::MX * 16, C::MX * 16, 128),
+                                              smem_desc(bd + (C::R / 8) * 128 + ks * 2 * C::NT * 16, C::NT * 16, 128),
+                                              idesc_g, 1u);
+                        }
 #pragma unroll
                         for (int ks = 0; ks < C::R / 16; ++ks)
                             tc_mma_f16_ss(tmem + C::DW_COL, smem_desc(bs + ks * 256, 128, C::R * 16),
@@ -760,9 +772,9 @@ __global__ void __launch_bounds__(BwdTcCfg<KS, NSL>::NTHREADS, 1) m2rnn_bwd_tc_k
     }
 }
 
-template <int KS, int NSL>
-static cudaError_t launch_bwd_tc_k(const Params& p0, cudaStream_t stream) {
-    using C = BwdTcCfg<KS, NSL>;
+template <int KS, int NSL, bool PAIR>
+static cudaError_t launch_bwd_tc_kp(const Params& p0, cudaStream_t stream) {
+    using C = BwdTcCfg<KS, NSL, PAIR>;
     static_assert(NSL <= 2, "slice partial sums are exact for two addends only");
     Params p = p0;
     p.dw_parts = NSL;   // one dW partial per slice
@@ -773,13 +785,23 @@ static cudaError_t launch_bwd_tc_k(const Params& p0, cudaStream_t stream) {
         e = cudaMemsetAsync(p.df, 0, sizeof(float) * (size_t)p.B * p.H * p.T, stream);
         if (e != cudaSuccess) return e;
     }
-    auto kern = m2rnn_bwd_tc_kernel<KS, NSL>;
+    auto kern = m2rnn_bwd_tc_kernel<KS, NSL, PAIR>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<p.B * p.H * NSL, C::NTHREADS, C::SMEM_BYTES, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     return launch_dw_reduce(p, stream);
+}
+
+// One bf16 dA operand up to T = 2048 steps, where it keeps every (b, h) pair of
+// three heads of the 410M training workload within 5.7e-3 of the oracle; the
+// compensated pair beyond, since the rounding of dA accumulates along the
+// reverse walk (at T = 4096 the single operand took a well-conditioned 7B-MoE
+// head from 3e-5 to 5e-3 on dk, one pair's df to 1.0e-2).
+template <int KS, int NSL>
+static cudaError_t launch_bwd_tc_k(const Params& p, cudaStream_t stream) {
+    return p.T > 2048 ? launch_bwd_tc_kp<KS, NSL, true>(p, stream) : launch_bwd_tc_kp<KS, NSL, false>(p, stream);
 }
 
 namespace {
